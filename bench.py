@@ -1,0 +1,517 @@
+"""Benchmark of the routed-experts forward on B200.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl b200|reference]
+
+One step = one ``moe_experts_forward`` call (dispatch tables + permute gather,
+grouped gate+up GEMM with the SwiGLU(+FP8) epilogue, grouped down GEMM,
+weighted unpermute, plus the shared expert where the workload has one) over one
+batch of seeded synthetic inputs already resident in HBM. L2 is flushed (a
+512 MiB write) before every timed step, outside the timed events. Each rank
+runs the same workload on its own GPU (weak scaling; the path needs no
+exchange). Rank 0 prints one JSON line.
+
+``--impl reference`` times the CPU oracle on the host cores on a bounded
+sample of the same workload (there is no installable reference program).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from moe_inputs import CONFIGS, get_config, make_hidden, make_logits, make_weights  # noqa: E402
+
+METRIC = "routed-experts fwd ms/layer + TFLOPS, % of B200 roofline (1 GPU)"
+DEFAULT_CONFIG = "qwen3_decode"
+# TileOPs PR #1580 (H200, bf16) experts-forward times for the same model families
+PAGE_MS = {"qwen3_decode": 3.219, "qwen3_prefill": 6.778, "dsv3_decode_fp8": None,
+           "dsv3_prefill": 9.465}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    d = dict(FALLBACK_PEAKS)
+    d["source"] = "fallback"
+    return d
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work: FLOPs 6*T*k*H*F (+ 6*T*H*F_s shared); bytes = touched experts'
+# weights + hidden in + out + ids/weights; intermediates are implementation traffic
+# ---------------------------------------------------------------------------
+
+def work_model(cfg, ids: np.ndarray) -> dict:
+    T, H, F, k = cfg.T, cfg.H, cfg.F, cfg.top_k
+    P = T * k
+    touched = int(np.unique(ids).size)
+    flops_routed = 6.0 * P * H * F
+    flops_shared = 6.0 * T * H * cfg.F_shared
+    w_gu = touched * 2 * F * H * 2
+    if cfg.down_fp8:
+        w_dn = touched * H * F * 1 + touched * (H // 128) * (F // 128) * 4
+    else:
+        w_dn = touched * H * F * 2
+    w_sh = (3 * H * cfg.F_shared * 2) if cfg.F_shared else 0
+    act = T * H * 2 * 2 + P * 8
+    total_bytes = w_gu + w_dn + w_sh + act
+    # gate+up kernel alone: its weights, its A rows (x_perm), its h output
+    gu_bytes = w_gu + P * H * 2 + P * F * (1 if cfg.down_fp8 else 2) + (P * (F // 128) * 4 if cfg.down_fp8 else 0)
+    dn_bytes = w_dn + P * F * (1 if cfg.down_fp8 else 2) + P * H * 2
+    return dict(touched=touched, flops=flops_routed + flops_shared, flops_routed=flops_routed,
+                bytes=total_bytes, gate_up_bytes=gu_bytes, gate_up_flops=4.0 * P * H * F,
+                down_bytes=dn_bytes, down_flops=2.0 * P * H * F)
+
+
+# ---------------------------------------------------------------------------
+# clocks
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append(dict(sm=float(parts[1]), smmax=float(parts[2]),
+                                     power=float(parts[3]) if parts[3] not in ("[N/A]", "") else 0.0,
+                                     hw=parts[5], hwt=parts[6], swt=parts[7], swp=parts[8]))
+                except ValueError:
+                    continue
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        pmax = max(r["power"] for r in rows)
+        loaded = [r for r in rows if r["power"] >= 0.5 * pmax] or rows
+        reasons = set()
+        for r in loaded:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("swp", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded),
+                "sm_max_mhz": max(r["smmax"] for r in rows), "reasons": sorted(reasons),
+                "samples": len(loaded)}
+
+
+# ---------------------------------------------------------------------------
+# the b200 arm
+# ---------------------------------------------------------------------------
+
+def build_layer(cfg, device):
+    import moe_routed_expert_top_b200 as M
+    from moe_routed_expert_top_b200.layer import RoutedExperts
+    w = make_weights(cfg, device)
+    layer = RoutedExperts(w["w_gate_up"], w["w_down"], cfg.top_k, cfg.score_fn, cfg.renormalize,
+                          cfg.routed_scaling_factor, cfg.down_fp8, w.get("ws_gate_up"),
+                          w.get("ws_down"))
+    del w
+    hidden = make_hidden(cfg, device)
+    logits = torch.from_numpy(make_logits(cfg)).to(device)
+    ids, weights = layer.route(logits)       # a1 on the GPU (bit-exact with the oracle)
+    torch.cuda.synchronize()
+    return M, layer, hidden, ids, weights, logits
+
+
+def time_steps(fn, steps, flush, stream):
+    """Per-step CUDA-event times (ms) of fn(), with an L2 flush before each."""
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        fn()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def stage_breakdown(M, layer, cfg, hidden, ids, weights, steps, flush):
+    """Device time of each stage launched alone through the C entry points on
+    the same workspace: tables+gather, gate+up GEMM, down GEMM, (shared), unpermute."""
+    prob = layer.problem(cfg.T)
+    T = cfg.T
+    ws = layer.workspace(T, hidden.device)
+    L = M.moe_get_tables_layout(prob)
+    dev = hidden.device
+    P = L["P"]
+    tables = torch.empty(L["total_int32"], dtype=torch.int32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    x_perm = torch.empty(P, cfg.H, dtype=torch.bfloat16, device=dev)
+    if cfg.down_fp8:
+        h = torch.empty(P, cfg.F, dtype=torch.uint8, device=dev)
+        hs = torch.empty(P, cfg.F // 128, dtype=torch.float32, device=dev)
+    else:
+        h = torch.empty(P, cfg.F, dtype=torch.bfloat16, device=dev)
+        hs = None
+    y = torch.empty(P, cfg.H, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(T, cfg.H, dtype=torch.bfloat16, device=dev)
+    addend = None
+    if cfg.F_shared:
+        sh = torch.empty(T, cfg.F_shared, dtype=torch.bfloat16, device=dev)
+        addend = torch.empty(T, cfg.H, dtype=torch.bfloat16, device=dev)
+    del ws
+    stages = {
+        "route_permute": lambda: M.moe_route_permute(prob, None, ids, None, hidden, x_perm,
+                                                     tables, status),
+        "gate_up_gemm": lambda: M.moe_grouped_gemm(
+            prob, 0, 2 * cfg.F, cfg.H, x_perm, None, layer.w_gate_up, None, tables,
+            M.MOE_EPI_SWIGLU_FP8 if cfg.down_fp8 else M.MOE_EPI_SWIGLU, h, hs, None, status),
+        "down_gemm": lambda: M.moe_grouped_gemm(
+            prob, 0, cfg.H, cfg.F, h, hs, layer.w_down, layer.w_down_scales, tables,
+            M.MOE_EPI_STORE, y, None, None, status),
+    }
+    if cfg.F_shared:
+        stages["shared_gate_up_gemm"] = lambda: M.moe_grouped_gemm(
+            None, T, 2 * cfg.F_shared, cfg.H, hidden, None, layer.ws_gate_up, None, None,
+            M.MOE_EPI_SWIGLU, sh, None, None, status)
+        stages["shared_down_gemm"] = lambda: M.moe_grouped_gemm(
+            None, T, cfg.H, cfg.F_shared, sh, None, layer.ws_down, None, None, M.MOE_EPI_STORE,
+            addend, None, None, status)
+    stages["unpermute"] = lambda: M.moe_unpermute(prob, y, tables, weights,
+                                                  cfg.routed_scaling_factor, addend, out)
+    stream = torch.cuda.current_stream()
+    res = {}
+    for name, fn in stages.items():
+        for _ in range(3):
+            fn()
+        ts = time_steps(fn, steps, flush, stream)
+        res[name] = statistics.median(ts)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    return res
+
+
+def run_b200(args, cfg, rank, world, device):
+    M, layer, hidden, ids, weights, logits = build_layer(cfg, device)
+    peaks = load_peaks()
+    wm = work_model(cfg, ids.cpu().numpy())
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+    out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        layer.forward(hidden, ids, weights, out)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0, "device status flag set"
+    launches_per_step = M.moe_last_launch_count()
+
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                      else int(os.environ.get("LOCAL_RANK", 0))) as clk:
+        t0 = time.perf_counter()
+        times = time_steps(step, args.steps, flush, stream)
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - t0
+    barrier(world)
+    ms = sum(times) / len(times)
+    ms = max_over_ranks(ms, world, device)
+    clocks = clk.summary()
+
+    # end to end through the public call with host buffers
+    hid_h = hidden.cpu().pin_memory()
+    ids_h = ids.cpu().pin_memory()
+    w_h = weights.cpu().pin_memory()
+    out_h = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16).pin_memory()
+    hid_d = torch.empty_like(hidden)
+    ids_d = torch.empty_like(ids)
+    w_d = torch.empty_like(weights)
+
+    def e2e_step():
+        hid_d.copy_(hid_h, non_blocking=True)
+        ids_d.copy_(ids_h, non_blocking=True)
+        w_d.copy_(w_h, non_blocking=True)
+        layer.forward(hid_d, ids_d, w_d, out)
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    e2e_times = time_steps(e2e_step, max(3, min(args.steps, 50)), flush, stream)
+    e2e_ms = max_over_ranks(sum(e2e_times) / len(e2e_times), world, device)
+
+    # stage breakdown and the dominant kernel's roofline
+    stages = stage_breakdown(M, layer, cfg, hidden, ids, weights, max(5, min(args.steps, 30)),
+                             flush)
+    dom = max(("gate_up_gemm", "down_gemm"), key=lambda s: stages[s])
+    dom_bytes = wm["gate_up_bytes"] if dom == "gate_up_gemm" else wm["down_bytes"]
+    dom_flops = wm["gate_up_flops"] if dom == "gate_up_gemm" else wm["down_flops"]
+    t_dom = stages[dom] * 1e-3
+    hbm = peaks["hbm_gbs"]
+    bf16 = peaks.get("bf16_tflops", 1590.0)
+    t_b = dom_bytes / (hbm * 1e9)
+    t_f = dom_flops / (bf16 * 1e12)
+    if t_b >= t_f:
+        roof = {"bound": "hbm", "achieved": round(dom_bytes / t_dom / 1e9, 1), "peak": hbm,
+                "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": round(dom_flops / t_dom / 1e12, 1), "peak": bf16,
+                "unit": "TFLOP/s"}
+    roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
+    roof["traffic"] = None
+    roof["kernel"] = dom
+    roof["peak_source"] = peaks["source"]
+
+    t_s = ms * 1e-3
+    t_flop = wm["flops"] / (bf16 * 1e12)
+    t_byte = wm["bytes"] / (hbm * 1e9)
+    fwd_roof = {"t_flop_us": round(t_flop * 1e6, 1), "t_byte_us": round(t_byte * 1e6, 1),
+                "frac": round(max(t_flop, t_byte) / t_s, 4),
+                "bound": "hbm" if t_byte >= t_flop else "tensor",
+                "algorithmic_bytes": wm["bytes"], "flops": wm["flops"],
+                "touched_experts": wm["touched"]}
+    tflops = world * wm["flops"] / t_s / 1e12
+    h2d = hidden.numel() * 2 + ids.numel() * 4 + weights.numel() * 4
+    d2h = out.numel() * 2
+    page = PAGE_MS.get(cfg.name)
+    line = {
+        "metric": METRIC, "value": round(ms, 4), "unit": "ms/layer", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": round(ms / page, 4) if page else None,
+        "tflops": round(tflops, 2), "dtype": "bf16+e4m3" if cfg.down_fp8 else "bf16",
+        "data": "synthetic",
+        "config": {"workload": cfg.name, "T": cfg.T, "E": cfg.E, "top_k": cfg.top_k, "H": cfg.H,
+                   "F": cfg.F, "F_shared": cfg.F_shared, "score_fn": cfg.score_fn,
+                   "routed_scaling_factor": cfg.routed_scaling_factor,
+                   "down_fp8": cfg.down_fp8, "l2": "flushed (512 MiB write) before each step",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": roof, "forward_roofline": fwd_roof,
+        "stages_ms": {k: round(v, 4) for k, v in stages.items()},
+        "e2e": {"value": round(e2e_ms, 4), "unit": "ms/layer", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks, "wall_s": round(wall, 3),
+    }
+    if rank == 0 and world == 1 and not args.skip_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, args.cpu_budget_s)
+    return line
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (baseline leg / reference arm)
+# ---------------------------------------------------------------------------
+
+class OracleRunner:
+    """The CPU oracle (as it stands) on the workload: routing and dispatch
+    tables over all tokens, then the per-token expert forward over a sample of
+    tokens. Weights are generated once (seeded N(0, 0.02) bf16 of the
+    workload's shapes; for the DeepSeek-size workloads, whose 22 GB of weights
+    would not fit a host comfortably, each expert the sample touches is drawn
+    when first needed and kept)."""
+
+    def __init__(self, cfg):
+        from oracle import moe_oracle as O
+        self.O = O
+        self.cfg = cfg
+        self.threads = torch.get_num_threads()
+        try:
+            import threadpoolctl
+            info = threadpoolctl.threadpool_info()
+            self.threads = max([i.get("num_threads", 1) for i in info] + [1])
+        except Exception:
+            pass
+        self.logits = make_logits(cfg)
+        self.hidden = make_hidden(cfg, "cpu")
+        small = cfg.E * cfg.H * cfg.F <= 600_000_000
+        self.weights = make_weights(cfg, "cpu") if small else None
+        self.cache = {}
+        self.shared = {}
+        if cfg.F_shared:
+            g = torch.Generator().manual_seed(7)
+            self.shared = dict(
+                ws_gate_up=(torch.randn(2 * cfg.F_shared, cfg.H, generator=g) * 0.02).to(torch.bfloat16),
+                ws_down=(torch.randn(cfg.H, cfg.F_shared, generator=g) * 0.02).to(torch.bfloat16))
+
+    def _loader(self, name, e):
+        if name not in ("w_gate_up", "w_down"):
+            return None
+        key = (name, int(e))
+        if key not in self.cache:
+            g = torch.Generator().manual_seed(2000 + 977 * int(e) + (name == "w_down"))
+            shape = (2 * self.cfg.F, self.cfg.H) if name == "w_gate_up" else (self.cfg.H, self.cfg.F)
+            self.cache[key] = (torch.randn(shape, generator=g) * 0.02).to(torch.bfloat16)
+        return self.cache[key]
+
+    def run(self, n: int) -> float:
+        """Seconds for one routed-experts forward of the first n tokens
+        (routing + tables over all T tokens)."""
+        O, cfg = self.O, self.cfg
+        t0 = time.perf_counter()
+        ids, w = O.route_topk(self.logits, cfg.top_k,
+                              O.SOFTMAX if cfg.score_fn == "softmax" else O.SIGMOID, cfg.renormalize)
+        O.dispatch_tables(ids, cfg.E, cfg.padding_M)
+        toks = np.arange(n)
+        if self.weights is not None:
+            O.experts_forward(self.hidden, ids, w, self.weights["w_gate_up"], self.weights["w_down"],
+                              cfg.routed_scaling_factor, tokens=toks, fp8=cfg.down_fp8, **self.shared)
+        else:
+            # draw the experts this sample touches (not timed)
+            t_gen = time.perf_counter()
+            for e in np.unique(ids[:n]):
+                self._loader("w_gate_up", e)
+                self._loader("w_down", e)
+            t0 += time.perf_counter() - t_gen
+            O.experts_forward(self.hidden, ids, w, None, None, cfg.routed_scaling_factor,
+                              tokens=toks, fp8=cfg.down_fp8, weight_loader=self._loader,
+                              **self.shared)
+        return time.perf_counter() - t0
+
+    def pick_sample(self, budget_s: float) -> int:
+        n = min(self.cfg.T, 8)
+        while n < self.cfg.T:
+            if self.run(n) > budget_s / 4:
+                break
+            n = min(self.cfg.T, n * 4)
+        return n
+
+    def describe(self, n: int) -> str:
+        return (f"{n} of {self.cfg.T} tokens through the per-token oracle (all their experts), "
+                f"time scaled by T/{n}; routing + dispatch tables on all {self.cfg.T} tokens")
+
+
+def cpu_baseline(cfg, budget_s: float = 20.0) -> dict:
+    r = OracleRunner(cfg)
+    n = r.pick_sample(budget_s)
+    t = r.run(n)
+    return {"value": round(t * cfg.T / n * 1e3, 1), "unit": "ms/layer", "cores": int(r.threads),
+            "kind": "oracle", "sample": r.describe(n), "sample_s": round(t, 2)}
+
+
+def run_reference(args, cfg) -> dict:
+    r = OracleRunner(cfg)
+    per_step = min(20.0, 150.0 / max(1, args.steps + args.warmup))
+    n = r.pick_sample(per_step * 4)
+    times = []
+    for i in range(args.warmup + args.steps):
+        t = r.run(n)
+        if i >= args.warmup:
+            times.append(t * cfg.T / n * 1e3)
+    v = round(statistics.median(times), 1)
+    return {"metric": METRIC, "value": v, "unit": "ms/layer", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": v,
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": cfg.name, "T": cfg.T, "E": cfg.E, "top_k": cfg.top_k,
+                       "H": cfg.H, "F": cfg.F},
+            "cpu_baseline": {"value": v, "unit": "ms/layer", "cores": int(r.threads),
+                             "kind": "oracle", "sample": r.describe(n)},
+            "e2e": {"value": v, "unit": "ms/layer", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int, device) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=list(CONFIGS))
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=20.0)
+    args = ap.parse_args(argv)
+    args.warmup = max(args.warmup, 3)
+    cfg = get_config(args.config)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, cfg)), flush=True)
+        return 0
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+    try:
+        from moe_routed_expert_top_b200 import build
+        build.build()
+        line = run_b200(args, cfg, rank, world, device)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,259 @@
+/*
+ * moe.h - C ABI of the B200 (sm_100a) routed mixture-of-experts expert forward.
+ *
+ * The library runs, on one GPU and on the caller's CUDA stream:
+ *   a1 top-k routing of router logits (softmax or sigmoid scores, optionally
+ *      renormalised over the k picks);
+ *   a2 the expert-sorted permutation and its dispatch tables (group_sizes,
+ *      group_offsets, group_padded_offsets, group_idx_for_bx) from one
+ *      histogram + stable scan kernel, with no host synchronisation;
+ *   a3 the permute gather of token rows into expert order;
+ *   a4 a persistent grouped gate+up GEMM on tcgen05 tensor cores (TMEM
+ *      accumulators, TMA loads whose out-of-bounds zero fill covers ragged
+ *      expert tails);
+ *   a5 SiLU(gate)*up in that GEMM's epilogue, optionally quantised to FP8
+ *      E4M3 with one fp32 scale per 1x128 tile;
+ *   a6 a grouped down GEMM, bf16 or FP8 with 128x128 block-scaled weights;
+ *   a7 a weighted unpermute that folds in routed_scaling_factor.
+ *
+ * Sources of the operations (web pages, cited by title and section):
+ *   [TUT07]  TileLang tutorial "Example 07: MoE dispatch contract and
+ *            quantised GEMM", section 1 (moe_dispatch_contract.py: the four
+ *            tables, m_start recovery, the 9-token example) and section 2
+ *            (skeletons.py: routed grouped GEMM -> SiLU -> down -> weighted
+ *            write-back).
+ *   [PR1580] TileOPs PR #1580 "Grouped-GEMM TMA OOB zero-fill + unpermute
+ *            out=": Grouped-GEMM kernel (C[e] = A[e] @ B[e]^T, A descriptor over
+ *            all rows, hardware zero fill of the partial last tile, no padding
+ *            copies or host sync) and Unpermute (out= buffer, scaling folded in
+ *            before the cast/store).
+ *   [PR778]  TileOPs PR #778 "SharedFusedMoE with native shared expert kernel
+ *            and TP support": Design (caller passes complete weights; merged
+ *            gate_up weight holds gate rows then up rows; shared expert
+ *            gate+up -> SiLU-mul -> down added to the routed output).
+ *   [PR2089] XTuner PR #2089 "Fuse MoE activation FP8 quantization kernels":
+ *            Changes (SiLU(gate)*up fused with W2-input 1x128 per-tile FP8
+ *            quantisation, no bf16 activation materialised).
+ *   [PR809]  pypto-lib PR #809 "predicate empty routed-expert stages": experts
+ *            with zero rows skip all compute.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller (PyTorch
+ *     supplies them). Row-major, densely packed, 16-byte aligned. bf16 values
+ *     are passed as `const void*` / `void*` (2 bytes each, IEEE bfloat16).
+ *   - The library never allocates, frees or synchronises. Every call only
+ *     enqueues work on `stream` (NULL = the legacy default stream); a return of
+ *     MOE_OK means "validated and enqueued".
+ *   - Synchronous errors (bad arguments, unsupported shapes, a CUDA launch
+ *     error) are returned as moe_status before or at launch.
+ *   - Errors only the device can see (an expert id outside [0, E), a pipeline
+ *     wait that exceeded its time limit) are OR-ed as MOE_DEV_* flags into the
+ *     caller's int32 `dev_status` word, to be read after the stream is
+ *     synchronised. Kernels never trap: an out-of-range id is skipped, a wait
+ *     that times out makes the kernel drain its in-flight copies, free its
+ *     tensor memory and return.
+ *   - Symbols: T tokens, k = top_k, E experts, H hidden size, F expert FFN size,
+ *     P = T*k (token, expert) pairs.
+ */
+#ifndef MOE_B200_MOE_H_
+#define MOE_B200_MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* moe_stream_t;
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = -1,   /* null pointer, negative size, misaligned pointer, bad enum */
+  MOE_ERR_UNSUPPORTED = -2,   /* shape outside what the kernels handle (see each call) */
+  MOE_ERR_WORKSPACE = -3,     /* workspace smaller than moe_workspace_bytes() */
+  MOE_ERR_CUDA = -4,          /* a CUDA runtime/driver call failed (message: moe_last_cuda_error) */
+  MOE_ERR_TIMEOUT = -5,       /* reported by moe_decode_device_status for MOE_DEV_TIMEOUT */
+  MOE_ERR_DEVICE_FLAG = -6    /* reported by moe_decode_device_status for other device flags */
+} moe_status;
+
+/* Flags OR-ed into the int32 device status word. */
+enum {
+  MOE_DEV_BAD_EXPERT_ID = 1,  /* a topk id outside [0, E): that pair was skipped */
+  MOE_DEV_TIMEOUT = 2,        /* a kernel's bounded wait ran out; its outputs are invalid */
+  MOE_DEV_BAD_TABLES = 4      /* group tables inconsistent with the GEMM's shape */
+};
+
+enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 };
+
+/* Epilogues of moe_grouped_gemm. */
+enum {
+  MOE_EPI_STORE = 0,       /* C bf16 [rows, N] = A @ B^T */
+  MOE_EPI_SWIGLU = 1,      /* C bf16 [rows, N/2] = SiLU(G[:, :N/2]) * G[:, N/2:] */
+  MOE_EPI_SWIGLU_FP8 = 2   /* C e4m3 [rows, N/2] + C_scales fp32 [rows, N/256] */
+};
+
+/* One MoE layer's shape and routing options. */
+typedef struct moe_problem {
+  int32_t T;            /* tokens (>= 0; 0 is a no-op) */
+  int32_t H;            /* hidden size: multiple of 64 (of 128 with down_fp8) */
+  int32_t F;            /* expert FFN size: multiple of 64 (of 128 with down_fp8) */
+  int32_t E;            /* routed experts, 1..1024 */
+  int32_t top_k;        /* 1..min(E, 32) */
+  int32_t padding_M;    /* group_padded_offsets alignment = M-block height
+                           ("block_token" in [TUT07]); the GEMMs need 128 */
+  int32_t score_fn;     /* MOE_SCORE_SOFTMAX or MOE_SCORE_SIGMOID */
+  int32_t renormalize;  /* 1: weights renormalised over the k picks */
+  float routed_scaling_factor; /* applied in the unpermute (a7), not in routing */
+  int32_t down_fp8;     /* 1: FP8 1x128 activations and 128x128 block-scaled down weights */
+  int32_t F_shared;     /* shared expert FFN size (multiple of 64), 0 = none */
+} moe_problem;
+
+/* Layout of the int32 dispatch-table buffer written by moe_route_permute.
+ * Offsets are in int32 elements from the buffer's start ([TUT07] section 1):
+ *   group_sizes[E]            pairs routed to each expert
+ *   group_offsets[E+1]        exclusive scan of sizes; [E] = P
+ *   group_padded_offsets[E+1] exclusive scan of ceil(size/padding_M)*padding_M
+ *   group_idx_for_bx[M_blk]   M-block -> expert: the largest g whose padded
+ *                             offset is <= bx*padding_M; M_blk = ceil(P/padding_M)+E
+ *   row_of_pair[P]            permuted row of flat pair p = t*k + j; experts in
+ *                             index order, pairs of one expert in flat order
+ *   pair_of_row[P]            inverse permutation (-1 for rows left empty by
+ *                             out-of-range ids) */
+typedef struct moe_tables_layout {
+  int64_t group_sizes;
+  int64_t group_offsets;
+  int64_t group_padded_offsets;
+  int64_t group_idx_for_bx;
+  int64_t row_of_pair;
+  int64_t pair_of_row;
+  int64_t total_int32;  /* elements the buffer must hold */
+  int32_t M_blk;
+  int32_t P;
+} moe_tables_layout;
+
+/* Fills *out for `prob`. Errors: MOE_ERR_INVALID_ARG for null or bad sizes. */
+moe_status moe_get_tables_layout(const moe_problem* prob, moe_tables_layout* out);
+
+/* Bytes of device workspace moe_experts_forward needs for `prob` (0 on a bad
+ * problem). The first 4 bytes of the workspace are the call's int32 device
+ * status word (see MOE_DEV_*); the rest holds the tables, the permuted rows,
+ * the SwiGLU output (bf16, or e4m3 codes + fp32 scales), the down output and
+ * the shared expert's intermediates, each 1024-byte aligned. */
+size_t moe_workspace_bytes(const moe_problem* prob);
+
+/* a1: top-k routing ([PR778] Benchmark: sigmoid routing for DeepSeek/Kimi-K2).
+ * logits fp32 [T, E] -> topk_ids int32 [T, k] (largest logit first; equal
+ * logits: lower expert index first) and topk_weights fp32 [T, k]:
+ *   softmax+renorm: w_j = e_j / sum_{i<k} e_i, e_j = exp(l_j - l_top1)
+ *   softmax:        w_j = exp(l_j - max l) / sum over all E (index order)
+ *   sigmoid:        s_j = 1/(1+exp(-l_j)); renorm w_j = s_j / sum_{i<k} s_i
+ * in float32 with a fixed exp (Cody-Waite reduction, degree-7 Taylor), sums
+ * in slot order, IEEE division: results are reproducible bit for bit.
+ * routed_scaling_factor is NOT applied here. */
+moe_status moe_route_topk(const moe_problem* prob, const float* logits,
+                          int32_t* topk_ids, float* topk_weights, moe_stream_t stream);
+
+/* a1 (optional) + a2 + a3 ([TUT07] section 1; [PR1580] no host sync).
+ * If `logits` is non-null, routes first (as moe_route_topk) into topk_ids /
+ * topk_weights; otherwise topk_ids [T, k] is an input and topk_weights unused.
+ * Writes the dispatch tables into `tables` (moe_tables_layout) and, if
+ * `hidden` [T, H] bf16 is non-null, x_perm [P, H] bf16 with
+ * x_perm[row_of_pair[p]] = hidden[p / k]. Any padding_M >= 1 is accepted.
+ * Device flags: MOE_DEV_BAD_EXPERT_ID into *dev_status (required). */
+moe_status moe_route_permute(const moe_problem* prob, const float* logits,
+                             int32_t* topk_ids, float* topk_weights,
+                             const void* hidden, void* x_perm, int32_t* tables,
+                             int32_t* dev_status, moe_stream_t stream);
+
+/* a4 / a6: grouped GEMM C = A @ B[e]^T over each expert's rows
+ * ([PR1580] Grouped-GEMM kernel), persistent, tcgen05 + TMEM + TMA.
+ *   tables non-null (grouped): A [P, K] rows in expert order (P = T*k of
+ *     `prob`), B [E, N, K]; M-block bx covers rows of expert group_idx_for_bx[bx]
+ *     (padding_M must be 128); experts with no rows are never scheduled.
+ *   tables null (dense, one group): A [M_rows, K], B [N, K].
+ * bf16 mode (A_scales == B_scales == NULL): A, B bf16; K % 64 == 0.
+ *   MOE_EPI_STORE:      C bf16 [rows, N], N % 64 == 0.
+ *   MOE_EPI_SWIGLU:     N = 2F with gate = B rows [0,F), up = rows [F,2F)
+ *                       ([PR778] Design); C bf16 [rows, F]; F % 64 == 0.
+ *   MOE_EPI_SWIGLU_FP8: as SWIGLU, then per row and 128-column tile
+ *                       s = amax/448, q = e4m3_rn_satfinite(h/s) (s = 0, q = 0
+ *                       for an all-zero tile) ([PR2089] Changes); C e4m3 codes
+ *                       [rows, F], C_scales fp32 [rows, F/128]; F % 128 == 0.
+ *                       debug_h (nullable) receives the fp32 h [rows, F].
+ * FP8 mode (A_scales and B_scales non-null): A e4m3 [rows, K] with A_scales
+ *   fp32 [rows, K/128]; B e4m3 [E, N, K] with B_scales fp32 [E, N/128, K/128];
+ *   C bf16 [rows, N] = sum over K-blocks kb of sa[r,kb]*sb[n/128,kb]*(A_kb @ B_kb^T);
+ *   epilogue must be MOE_EPI_STORE; N % 128 == 0, K % 128 == 0.
+ * Device flags: MOE_DEV_TIMEOUT into *dev_status (required). */
+moe_status moe_grouped_gemm(const moe_problem* prob, int32_t M_rows, int32_t N, int32_t K,
+                            const void* A, const float* A_scales,
+                            const void* B, const float* B_scales,
+                            const int32_t* tables, int32_t epilogue,
+                            void* C, float* C_scales, float* debug_h,
+                            int32_t* dev_status, moe_stream_t stream);
+
+/* a5 standalone ([PR2089] Changes): SwiGLU and/or 1x128 FP8 quantisation.
+ *   gate_up bf16 [M, 2F] non-null: h = SiLU(gate_up[:, :F]) * gate_up[:, F:]
+ *     in fp32; out_fp8 == 0 -> out bf16 [M, F] (round to nearest even);
+ *     out_fp8 == 1 -> out e4m3 [M, F] + scales fp32 [M, ceil(F/128)].
+ *   gate_up NULL, h fp32 [M, F] non-null: quantise h (out_fp8 must be 1).
+ * Quantisation rule as MOE_EPI_SWIGLU_FP8; a partial last tile takes amax
+ * over its valid columns. F % 4 == 0. */
+moe_status moe_swiglu_quant(int32_t M, int32_t F, const void* gate_up, const float* h,
+                            int32_t out_fp8, void* out, float* scales, moe_stream_t stream);
+
+/* a7 ([PR1580] Unpermute): out bf16 [T, H] =
+ *   RNE_bf16( scale * sum_{j<k} topk_weights[t,j] * y[row_of_pair[t*k+j]] + addend[t] )
+ * with the sum in fp32 in slot order j; y bf16 [P, H]; addend bf16 [T, H] or
+ * NULL; tables as written by moe_route_permute (row -1 contributes nothing). */
+moe_status moe_unpermute(const moe_problem* prob, const void* y, const int32_t* tables,
+                         const float* topk_weights, float scale, const void* addend,
+                         void* out, moe_stream_t stream);
+
+/* Offline weight preparation for the FP8 down GEMM: for each of `batch`
+ * matrices w bf16 [N, K], per 128x128 block s = amax/448 and
+ * q = e4m3_rn_satfinite(w/s) (all-zero block: s = 0, q = 0); q uint8
+ * [batch, N, K], scales fp32 [batch, ceil(N/128), ceil(K/128)]. */
+moe_status moe_quantize_weight_128x128(int32_t batch, int32_t N, int32_t K, const void* w,
+                                       uint8_t* q, float* scales, moe_stream_t stream);
+
+/* The whole routed-experts forward (a2..a7, plus the shared expert when
+ * prob->F_shared > 0): from given topk_ids / topk_weights [T, k],
+ *   out bf16 [T, H] = RNE_bf16( scale * sum_j w[t,j] * MLP_{e(t,j)}(hidden[t])
+ *                               + shared_MLP(hidden[t]) )
+ * with MLP_e(x) = W_down[e] (bf16(SiLU(G_gate) * G_up)), G = W_gate_up[e] x.
+ *   w_gate_up bf16 [E, 2F, H]; w_down bf16 [E, H, F], or with prob->down_fp8
+ *   e4m3 [E, H, F] plus w_down_scales fp32 [E, H/128, F/128] (see
+ *   moe_quantize_weight_128x128); ws_gate_up bf16 [2F_s, H], ws_down bf16
+ *   [H, F_s] when F_shared > 0 (else NULL).
+ * Needs prob->padding_M == 128. `workspace` (ws_bytes >= moe_workspace_bytes)
+ * is caller-owned device memory; its first int32 is this call's device status
+ * (zeroed by the call, then OR-ed with MOE_DEV_* flags). */
+moe_status moe_experts_forward(const moe_problem* prob, const void* hidden,
+                               const int32_t* topk_ids, const float* topk_weights,
+                               const void* w_gate_up, const void* w_down,
+                               const float* w_down_scales,
+                               const void* ws_gate_up, const void* ws_down,
+                               float scale, void* out, void* workspace, size_t ws_bytes,
+                               moe_stream_t stream);
+
+/* Maps a device status word (copied to the host after a sync) to a status:
+ * MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_DEVICE_FLAG. */
+moe_status moe_decode_device_status(int32_t dev_status);
+
+/* Static, human-readable name of a status. */
+const char* moe_status_string(moe_status status);
+
+/* Text of the last CUDA error seen by this thread's calls ("" if none). */
+const char* moe_last_cuda_error(void);
+
+/* Kernels the last moe_experts_forward call on this thread enqueued. */
+int32_t moe_last_launch_count(void);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* MOE_B200_MOE_H_ */

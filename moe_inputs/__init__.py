@@ -78,8 +78,9 @@ CONFIGS = {
 }
 
 
-def get_config(name: str, **overrides) -> MoeConfig:
-    cfg = CONFIGS[name]
+def get_config(config_name: str, **overrides) -> MoeConfig:
+    """A named workload, optionally with fields replaced (``name`` included)."""
+    cfg = CONFIGS[config_name]
     return cfg.replace(**overrides) if overrides else cfg
 
 

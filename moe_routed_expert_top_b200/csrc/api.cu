@@ -1,0 +1,406 @@
+// api.cu - the extern "C" entry points declared in include/moe.h: argument
+// validation, table/workspace layout, and the launch sequence of the whole
+// routed-experts forward. No allocation, no host synchronisation: every call
+// only enqueues kernels on the caller's stream.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "internal.h"
+#include "moe.h"
+
+namespace {
+
+thread_local char g_last_error[256] = "";
+thread_local int32_t g_last_launches = 0;
+
+moe_status cuda_fail(cudaError_t e) {
+  std::strncpy(g_last_error, cudaGetErrorString(e), sizeof(g_last_error) - 1);
+  g_last_error[sizeof(g_last_error) - 1] = '\0';
+  return MOE_ERR_CUDA;
+}
+
+#define MOE_CUDA_TRY(expr)                  \
+  do {                                      \
+    cudaError_t _e = (expr);                \
+    if (_e != cudaSuccess) return cuda_fail(_e); \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int64_t kMaxPairs = (1ll << 31) - (1ll << 20);
+
+// Shape rules shared by every call that takes a moe_problem.
+moe_status check_problem(const moe_problem* pr, bool need_gemm) {
+  if (pr == nullptr) return MOE_ERR_INVALID_ARG;
+  if (pr->T < 0 || pr->H <= 0 || pr->F <= 0 || pr->E <= 0 || pr->top_k <= 0 ||
+      pr->padding_M <= 0 || pr->F_shared < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (pr->score_fn != MOE_SCORE_SOFTMAX && pr->score_fn != MOE_SCORE_SIGMOID)
+    return MOE_ERR_INVALID_ARG;
+  if (pr->E > 1024 || pr->top_k > 32 || pr->top_k > pr->E) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(pr->T) * pr->top_k > kMaxPairs) return MOE_ERR_UNSUPPORTED;
+  if (pr->padding_M > (1 << 20)) return MOE_ERR_UNSUPPORTED;
+  if (need_gemm) {
+    if (pr->padding_M != 128) return MOE_ERR_UNSUPPORTED;
+    if (pr->H % 64 != 0 || pr->F % 64 != 0 || pr->F_shared % 64 != 0) return MOE_ERR_UNSUPPORTED;
+    if (pr->down_fp8 && (pr->H % 128 != 0 || pr->F % 128 != 0)) return MOE_ERR_UNSUPPORTED;
+  }
+  return MOE_OK;
+}
+
+int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
+
+void fill_layout(const moe_problem* pr, moe_tables_layout* L) {
+  const int64_t E = pr->E;
+  const int64_t P = static_cast<int64_t>(pr->T) * pr->top_k;
+  const int64_t M_blk = (P + pr->padding_M - 1) / pr->padding_M + E;
+  int64_t o = 0;
+  L->group_sizes = o;
+  o += round_up(E, 4);
+  L->group_offsets = o;
+  o += round_up(E + 1, 4);
+  L->group_padded_offsets = o;
+  o += round_up(E + 1, 4);
+  L->group_idx_for_bx = o;
+  o += round_up(M_blk, 4);
+  L->row_of_pair = o;
+  o += round_up(P, 4);
+  L->pair_of_row = o;
+  o += round_up(P, 4);
+  L->total_int32 = o;
+  L->M_blk = static_cast<int32_t>(M_blk);
+  L->P = static_cast<int32_t>(P);
+}
+
+struct WorkspacePlan {
+  int64_t status = 0, tables = 0, x_perm = 0, h = 0, h_scales = 0, y = 0, hs = 0, ys = 0, total = 0;
+};
+
+WorkspacePlan plan_workspace(const moe_problem* pr) {
+  moe_tables_layout L;
+  fill_layout(pr, &L);
+  const int64_t P = L.P, T = pr->T, H = pr->H, F = pr->F, Fs = pr->F_shared;
+  WorkspacePlan w;
+  int64_t o = 0;
+  auto take = [&](int64_t bytes) {
+    const int64_t at = o;
+    o = round_up(o + bytes, 1024);
+    return at;
+  };
+  w.status = take(256);
+  w.tables = take(L.total_int32 * 4);
+  w.x_perm = take(P * H * 2);
+  w.h = take(P * F * (pr->down_fp8 ? 1 : 2));
+  w.h_scales = take(pr->down_fp8 ? P * (F / 128) * 4 : 0);
+  w.y = take(P * H * 2);
+  w.hs = take(Fs ? T * Fs * 2 : 0);
+  w.ys = take(Fs ? T * H * 2 : 0);
+  w.total = o;
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_get_tables_layout(const moe_problem* prob, moe_tables_layout* out) {
+  if (out == nullptr) return MOE_ERR_INVALID_ARG;
+  const moe_status s = check_problem(prob, false);
+  if (s != MOE_OK) return s;
+  fill_layout(prob, out);
+  return MOE_OK;
+}
+
+size_t moe_workspace_bytes(const moe_problem* prob) {
+  if (check_problem(prob, true) != MOE_OK) return 0;
+  return static_cast<size_t>(plan_workspace(prob).total);
+}
+
+moe_status moe_route_topk(const moe_problem* prob, const float* logits, int32_t* topk_ids,
+                          float* topk_weights, moe_stream_t stream) {
+  moe_status s = check_problem(prob, false);
+  if (s != MOE_OK) return s;
+  if (prob->T == 0) return MOE_OK;
+  if (logits == nullptr || topk_ids == nullptr || topk_weights == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  MOE_CUDA_TRY(moe::launch_route_topk(logits, prob->T, prob->E, prob->top_k, prob->score_fn,
+                                      prob->renormalize, topk_ids, topk_weights,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_route_permute(const moe_problem* prob, const float* logits, int32_t* topk_ids,
+                             float* topk_weights, const void* hidden, void* x_perm,
+                             int32_t* tables, int32_t* dev_status, moe_stream_t stream) {
+  moe_status s = check_problem(prob, false);
+  if (s != MOE_OK) return s;
+  if (prob->T == 0) return MOE_OK;
+  if (topk_ids == nullptr || tables == nullptr || dev_status == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (logits != nullptr && topk_weights == nullptr) return MOE_ERR_INVALID_ARG;
+  if (hidden != nullptr && (x_perm == nullptr || !aligned16(hidden) || !aligned16(x_perm) ||
+                            prob->H % 8 != 0))
+    return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  moe_tables_layout L;
+  fill_layout(prob, &L);
+  if (logits != nullptr)
+    MOE_CUDA_TRY(moe::launch_route_topk(logits, prob->T, prob->E, prob->top_k, prob->score_fn,
+                                        prob->renormalize, topk_ids, topk_weights, st));
+  MOE_CUDA_TRY(moe::launch_tables(topk_ids, L.P, prob->E, prob->padding_M, L.M_blk,
+                                  tables + L.group_sizes, tables + L.group_offsets,
+                                  tables + L.group_padded_offsets, tables + L.group_idx_for_bx,
+                                  tables + L.row_of_pair, tables + L.pair_of_row, dev_status, st));
+  if (hidden != nullptr)
+    MOE_CUDA_TRY(moe::launch_gather_rows(hidden, tables + L.pair_of_row, L.P, prob->top_k,
+                                         prob->H, x_perm, st));
+  return MOE_OK;
+}
+
+moe_status moe_grouped_gemm(const moe_problem* prob, int32_t M_rows, int32_t N, int32_t K,
+                            const void* A, const float* A_scales, const void* B,
+                            const float* B_scales, const int32_t* tables, int32_t epilogue,
+                            void* C, float* C_scales, float* debug_h, int32_t* dev_status,
+                            moe_stream_t stream) {
+  if (A == nullptr || B == nullptr || C == nullptr || dev_status == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (N <= 0 || K <= 0) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(C)) return MOE_ERR_INVALID_ARG;
+  const bool fp8 = A_scales != nullptr || B_scales != nullptr;
+  if (fp8 && (A_scales == nullptr || B_scales == nullptr)) return MOE_ERR_INVALID_ARG;
+  moe::GemmLaunch g;
+  if (tables != nullptr) {
+    moe_status s = check_problem(prob, false);
+    if (s != MOE_OK) return s;
+    if (prob->padding_M != 128) return MOE_ERR_UNSUPPORTED;
+    moe_tables_layout L;
+    fill_layout(prob, &L);
+    g.rows = L.P;
+    g.E = prob->E;
+    g.group_sizes = tables + L.group_sizes;
+    g.group_offsets = tables + L.group_offsets;
+    g.group_padded = tables + L.group_padded_offsets;
+    g.idx_for_bx = tables + L.group_idx_for_bx;
+    g.M_blk = L.M_blk;
+  } else {
+    if (M_rows < 0) return MOE_ERR_INVALID_ARG;
+    g.rows = M_rows;
+    g.E = 1;
+  }
+  if (g.rows == 0) return MOE_OK;
+  if (fp8) {
+    if (epilogue != MOE_EPI_STORE) return MOE_ERR_UNSUPPORTED;
+    if (N % 128 != 0 || K % 128 != 0) return MOE_ERR_UNSUPPORTED;
+    g.mode = moe::kModeFp8Store;
+  } else {
+    if (K % 64 != 0) return MOE_ERR_UNSUPPORTED;
+    switch (epilogue) {
+      case MOE_EPI_STORE:
+        if (N % 64 != 0) return MOE_ERR_UNSUPPORTED;
+        g.mode = moe::kModeStore;
+        break;
+      case MOE_EPI_SWIGLU:
+        if (N % 128 != 0) return MOE_ERR_UNSUPPORTED;  // F = N/2 multiple of 64
+        g.mode = moe::kModeSwiglu;
+        break;
+      case MOE_EPI_SWIGLU_FP8:
+        if (N % 256 != 0) return MOE_ERR_UNSUPPORTED;  // F multiple of 128
+        if (C_scales == nullptr) return MOE_ERR_INVALID_ARG;
+        if (debug_h != nullptr && !aligned16(debug_h)) return MOE_ERR_INVALID_ARG;
+        g.mode = moe::kModeSwigluFp8;
+        break;
+      default:
+        return MOE_ERR_INVALID_ARG;
+    }
+  }
+  g.N = N;
+  g.K = K;
+  g.A = A;
+  g.B = B;
+  g.A_scales = A_scales;
+  g.B_scales = B_scales;
+  g.C = C;
+  g.C_scales = C_scales;
+  g.debug_h = debug_h;
+  g.status = dev_status;
+  MOE_CUDA_TRY(moe::launch_grouped_gemm(g, reinterpret_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_swiglu_quant(int32_t M, int32_t F, const void* gate_up, const float* h,
+                            int32_t out_fp8, void* out, float* scales, moe_stream_t stream) {
+  if (M < 0 || F <= 0 || F % 4 != 0) return MOE_ERR_INVALID_ARG;
+  if (M == 0) return MOE_OK;
+  if (out == nullptr) return MOE_ERR_INVALID_ARG;
+  if ((gate_up == nullptr) == (h == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (gate_up == nullptr && !out_fp8) return MOE_ERR_INVALID_ARG;
+  if (out_fp8 && scales == nullptr) return MOE_ERR_INVALID_ARG;
+  if ((gate_up && !aligned16(gate_up)) || (h && !aligned16(h)) || !aligned16(out))
+    return MOE_ERR_INVALID_ARG;
+  MOE_CUDA_TRY(moe::launch_swiglu_quant(M, F, gate_up, h, out_fp8 ? 1 : 0, out, scales,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_unpermute(const moe_problem* prob, const void* y, const int32_t* tables,
+                         const float* topk_weights, float scale, const void* addend, void* out,
+                         moe_stream_t stream) {
+  moe_status s = check_problem(prob, false);
+  if (s != MOE_OK) return s;
+  if (prob->T == 0) return MOE_OK;
+  if (y == nullptr || tables == nullptr || topk_weights == nullptr || out == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (prob->H % 8 != 0 || !aligned16(y) || !aligned16(out) || (addend && !aligned16(addend)))
+    return MOE_ERR_INVALID_ARG;
+  moe_tables_layout L;
+  fill_layout(prob, &L);
+  MOE_CUDA_TRY(moe::launch_unpermute(y, tables + L.row_of_pair, topk_weights, prob->T,
+                                     prob->top_k, prob->H, scale, addend, out,
+                                     reinterpret_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_quantize_weight_128x128(int32_t batch, int32_t N, int32_t K, const void* w,
+                                       uint8_t* q, float* scales, moe_stream_t stream) {
+  if (batch < 0 || N < 0 || K < 0 || w == nullptr || q == nullptr || scales == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (N % 128 != 0 || K % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (batch > 65535 || N / 128 > 65535) return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(w) || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+  MOE_CUDA_TRY(moe::launch_quantize_weight(batch, N, K, w, q, scales,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_experts_forward(const moe_problem* prob, const void* hidden,
+                               const int32_t* topk_ids, const float* topk_weights,
+                               const void* w_gate_up, const void* w_down,
+                               const float* w_down_scales, const void* ws_gate_up,
+                               const void* ws_down, float scale, void* out, void* workspace,
+                               size_t ws_bytes, moe_stream_t stream) {
+  g_last_launches = 0;
+  moe_status s = check_problem(prob, true);
+  if (s != MOE_OK) return s;
+  if (prob->T == 0) return MOE_OK;
+  if (hidden == nullptr || topk_ids == nullptr || topk_weights == nullptr ||
+      w_gate_up == nullptr || w_down == nullptr || out == nullptr || workspace == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (prob->down_fp8 && w_down_scales == nullptr) return MOE_ERR_INVALID_ARG;
+  if (prob->F_shared > 0 && (ws_gate_up == nullptr || ws_down == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(hidden) || !aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(out) ||
+      !aligned16(workspace) || (ws_gate_up && !aligned16(ws_gate_up)) ||
+      (ws_down && !aligned16(ws_down)))
+    return MOE_ERR_INVALID_ARG;
+  const WorkspacePlan w = plan_workspace(prob);
+  if (ws_bytes < static_cast<size_t>(w.total)) return MOE_ERR_WORKSPACE;
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  int32_t* status = reinterpret_cast<int32_t*>(base + w.status);
+  int32_t* tables = reinterpret_cast<int32_t*>(base + w.tables);
+  void* x_perm = base + w.x_perm;
+  void* h = base + w.h;
+  float* h_scales = reinterpret_cast<float*>(base + w.h_scales);
+  void* y = base + w.y;
+  moe_tables_layout L;
+  fill_layout(prob, &L);
+  const int T = prob->T, H = prob->H, F = prob->F, E = prob->E, k = prob->top_k;
+
+  MOE_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int32_t), st));
+  // a2 + a3
+  MOE_CUDA_TRY(moe::launch_tables(topk_ids, L.P, E, prob->padding_M, L.M_blk,
+                                  tables + L.group_sizes, tables + L.group_offsets,
+                                  tables + L.group_padded_offsets, tables + L.group_idx_for_bx,
+                                  tables + L.row_of_pair, tables + L.pair_of_row, status, st));
+  MOE_CUDA_TRY(moe::launch_gather_rows(hidden, tables + L.pair_of_row, L.P, k, H, x_perm, st));
+  g_last_launches += 2;
+
+  moe::GemmLaunch g;
+  g.rows = L.P;
+  g.E = E;
+  g.group_sizes = tables + L.group_sizes;
+  g.group_offsets = tables + L.group_offsets;
+  g.group_padded = tables + L.group_padded_offsets;
+  g.idx_for_bx = tables + L.group_idx_for_bx;
+  g.M_blk = L.M_blk;
+  g.status = status;
+  // a4 + a5: gate+up with the SwiGLU (+ FP8 1x128) epilogue
+  g.mode = prob->down_fp8 ? moe::kModeSwigluFp8 : moe::kModeSwiglu;
+  g.N = 2 * F;
+  g.K = H;
+  g.A = x_perm;
+  g.B = w_gate_up;
+  g.C = h;
+  g.C_scales = prob->down_fp8 ? h_scales : nullptr;
+  MOE_CUDA_TRY(moe::launch_grouped_gemm(g, st));
+  // a6: down
+  g.mode = prob->down_fp8 ? moe::kModeFp8Store : moe::kModeStore;
+  g.N = H;
+  g.K = F;
+  g.A = h;
+  g.B = w_down;
+  g.A_scales = prob->down_fp8 ? h_scales : nullptr;
+  g.B_scales = prob->down_fp8 ? w_down_scales : nullptr;
+  g.C = y;
+  g.C_scales = nullptr;
+  MOE_CUDA_TRY(moe::launch_grouped_gemm(g, st));
+  g_last_launches += 2;
+
+  // shared expert: a dense SwiGLU MLP on all tokens, added in the unpermute
+  const void* addend = nullptr;
+  if (prob->F_shared > 0) {
+    moe::GemmLaunch d;
+    d.rows = T;
+    d.E = 1;
+    d.status = status;
+    d.mode = moe::kModeSwiglu;
+    d.N = 2 * prob->F_shared;
+    d.K = H;
+    d.A = hidden;
+    d.B = ws_gate_up;
+    d.C = base + w.hs;
+    MOE_CUDA_TRY(moe::launch_grouped_gemm(d, st));
+    d.mode = moe::kModeStore;
+    d.N = H;
+    d.K = prob->F_shared;
+    d.A = base + w.hs;
+    d.B = ws_down;
+    d.C = base + w.ys;
+    MOE_CUDA_TRY(moe::launch_grouped_gemm(d, st));
+    addend = base + w.ys;
+    g_last_launches += 2;
+  }
+  // a7
+  MOE_CUDA_TRY(moe::launch_unpermute(y, tables + L.row_of_pair, topk_weights, T, k, H, scale,
+                                     addend, out, st));
+  g_last_launches += 1;
+  return MOE_OK;
+}
+
+moe_status moe_decode_device_status(int32_t dev_status) {
+  if (dev_status == 0) return MOE_OK;
+  if (dev_status & MOE_DEV_TIMEOUT) return MOE_ERR_TIMEOUT;
+  return MOE_ERR_DEVICE_FLAG;
+}
+
+const char* moe_status_string(moe_status status) {
+  switch (status) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+    case MOE_ERR_DEVICE_FLAG: return "MOE_ERR_DEVICE_FLAG";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+const char* moe_last_cuda_error(void) { return g_last_error; }
+
+int32_t moe_last_launch_count(void) { return g_last_launches; }
+
+}  // extern "C"

@@ -1,0 +1,207 @@
+// elementwise.cu - a7 weighted unpermute, a5 standalone SwiGLU(+E4M3 1x128
+// quantisation), and the offline 128x128 block quantisation of FP8 weights.
+// All three are HBM-streaming kernels: 16-byte vector loads/stores, fp32 math.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace moe {
+
+// ---------------------------------------------------------------------------
+// a7: out[t] = bf16( scale * sum_j w[t,j] * y[row_of_pair[t*k+j]] + addend[t] )
+// (TileOPs PR #1580, Unpermute: scaling folded in before the cast/store; the
+// result is written straight into the caller's output buffer). One thread per
+// 8 columns of one token; fp32 accumulation in slot order j.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) unpermute_kernel(const uint4* __restrict__ y,
+                                                        const int32_t* __restrict__ row_of_pair,
+                                                        const float* __restrict__ w, int k,
+                                                        int P, int H8, float scale,
+                                                        const uint4* __restrict__ addend,
+                                                        uint4* __restrict__ out) {
+  const int t = blockIdx.y;
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= H8) return;
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+  const int64_t pbase = static_cast<int64_t>(t) * k;
+  for (int j = 0; j < k; ++j) {
+    const int row = __ldg(row_of_pair + pbase + j);
+    if (row < 0 || row >= P) continue;
+    const float wt = __ldg(w + pbase + j);
+    const uint4 v = __ldg(y + static_cast<int64_t>(row) * H8 + c);
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc[2 * i] = fmaf(wt, bf16lo_to_f32(u[i]), acc[2 * i]);
+      acc[2 * i + 1] = fmaf(wt, bf16hi_to_f32(u[i]), acc[2 * i + 1]);
+    }
+  }
+  uint32_t o[4];
+  if (addend != nullptr) {
+    const uint4 a = __ldg(addend + static_cast<int64_t>(t) * H8 + c);
+    const uint32_t au[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      o[i] = pack_bf16x2(fmaf(scale, acc[2 * i], bf16lo_to_f32(au[i])),
+                         fmaf(scale, acc[2 * i + 1], bf16hi_to_f32(au[i])));
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] = pack_bf16x2(scale * acc[2 * i], scale * acc[2 * i + 1]);
+  }
+  out[static_cast<int64_t>(t) * H8 + c] = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+cudaError_t launch_unpermute(const void* y, const int32_t* row_of_pair, const float* weights,
+                             int T, int k, int H, float scale, const void* addend, void* out,
+                             cudaStream_t stream) {
+  if (T <= 0) return cudaSuccess;
+  const int H8 = H / 8;
+  dim3 grid((H8 + 127) / 128, T);
+  unpermute_kernel<<<grid, 128, 0, stream>>>(static_cast<const uint4*>(y), row_of_pair, weights, k,
+                                             T * k, H8, scale, static_cast<const uint4*>(addend),
+                                             static_cast<uint4*>(out));
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// a5 standalone: h = SiLU(gate) * up (XTuner PR #2089, Changes), stored as
+// bf16, or quantised per row and 128-column tile: s = amax/448,
+// q = e4m3_rn_satfinite(h/s), s = 0 and q = 0 for an all-zero tile. One warp
+// per (row, tile), 4 columns per lane.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) swiglu_quant_kernel(int M, int F,
+                                                           const __nv_bfloat16* __restrict__ gu,
+                                                           const float* __restrict__ hin,
+                                                           int out_fp8, void* __restrict__ out,
+                                                           float* __restrict__ scales) {
+  const int ntiles = (F + 127) / 128;
+  const long long gw = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (gw >= static_cast<long long>(M) * ntiles) return;
+  const int r = static_cast<int>(gw / ntiles);
+  const int tile = static_cast<int>(gw - static_cast<long long>(r) * ntiles);
+  const int col = tile * 128 + lane * 4;
+  const bool active = col < F;  // F % 4 == 0: all four columns valid or none
+  float h[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  if (active) {
+    if (gu != nullptr) {
+      const uint2 gv = *reinterpret_cast<const uint2*>(gu + static_cast<int64_t>(r) * 2 * F + col);
+      const uint2 uv =
+          *reinterpret_cast<const uint2*>(gu + static_cast<int64_t>(r) * 2 * F + F + col);
+      const float g[4] = {bf16lo_to_f32(gv.x), bf16hi_to_f32(gv.x), bf16lo_to_f32(gv.y),
+                          bf16hi_to_f32(gv.y)};
+      const float u[4] = {bf16lo_to_f32(uv.x), bf16hi_to_f32(uv.x), bf16lo_to_f32(uv.y),
+                          bf16hi_to_f32(uv.y)};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) h[i] = g[i] / (1.0f + expf(-g[i])) * u[i];
+    } else {
+      const float4 v = *reinterpret_cast<const float4*>(hin + static_cast<int64_t>(r) * F + col);
+      h[0] = v.x;
+      h[1] = v.y;
+      h[2] = v.z;
+      h[3] = v.w;
+    }
+  }
+  if (!out_fp8) {
+    if (active) {
+      uint2 o = make_uint2(pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]));
+      *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out) + static_cast<int64_t>(r) * F +
+                                col) = o;
+    }
+    return;
+  }
+  float amax = fmaxf(fmaxf(fabsf(h[0]), fabsf(h[1])), fmaxf(fabsf(h[2]), fabsf(h[3])));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  const float s = amax / 448.0f;
+  if (active) {
+    uint32_t code = 0;
+    if (amax > 0.0f)
+      code = static_cast<uint32_t>(cvt_e4m3x2(h[0] / s, h[1] / s)) |
+             (static_cast<uint32_t>(cvt_e4m3x2(h[2] / s, h[3] / s)) << 16);
+    *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(out) + static_cast<int64_t>(r) * F + col) =
+        code;
+  }
+  if (lane == 0) scales[static_cast<int64_t>(r) * ntiles + tile] = amax > 0.0f ? s : 0.0f;
+}
+
+cudaError_t launch_swiglu_quant(int M, int F, const void* gate_up, const float* h, int out_fp8,
+                                void* out, float* scales, cudaStream_t stream) {
+  if (M <= 0 || F <= 0) return cudaSuccess;
+  const long long warps = static_cast<long long>(M) * ((F + 127) / 128);
+  const long long blocks = (warps + 7) / 8;
+  swiglu_quant_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+      M, F, static_cast<const __nv_bfloat16*>(gate_up), h, out_fp8, out, scales);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// 128x128 block quantisation of weights w [batch, N, K] (bf16) to E4M3 codes
+// and fp32 block scales. One CTA per block; thread i handles row i/2,
+// columns (i%2)*64 .. +64.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) quant_weight_kernel(const uint4* __restrict__ w, int N,
+                                                           int K, uint8_t* __restrict__ q,
+                                                           float* __restrict__ scales) {
+  const int kb = blockIdx.x, nb = blockIdx.y, b = blockIdx.z;
+  const int nbk = K / 128, nbn = N / 128;
+  const int tid = threadIdx.x;
+  const int r = nb * 128 + (tid >> 1);
+  const int c0 = kb * 128 + (tid & 1) * 64;
+  const int64_t base = (static_cast<int64_t>(b) * N + r) * K + c0;  // element index
+  const uint4* src = w + base / 8;
+  float v[64];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint4 x = __ldg(src + i);
+    const uint32_t u[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[8 * i + 2 * j] = bf16lo_to_f32(u[j]);
+      v[8 * i + 2 * j + 1] = bf16hi_to_f32(u[j]);
+    }
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fabsf(v[i]));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  __shared__ float s_max[8];
+  if ((tid & 31) == 0) s_max[tid >> 5] = amax;
+  __syncthreads();
+  amax = s_max[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) amax = fmaxf(amax, s_max[i]);
+  const float s = amax / 448.0f;
+  uint4* dst = reinterpret_cast<uint4*>(q + base);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t wd[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float* x = v + 16 * i + 4 * j;
+      wd[j] = amax > 0.0f ? (static_cast<uint32_t>(cvt_e4m3x2(x[0] / s, x[1] / s)) |
+                             (static_cast<uint32_t>(cvt_e4m3x2(x[2] / s, x[3] / s)) << 16))
+                          : 0u;
+    }
+    dst[i] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+  }
+  if (tid == 0)
+    scales[(static_cast<int64_t>(b) * nbn + nb) * nbk + kb] = amax > 0.0f ? s : 0.0f;
+}
+
+cudaError_t launch_quantize_weight(int batch, int N, int K, const void* w, uint8_t* q,
+                                   float* scales, cudaStream_t stream) {
+  if (batch <= 0 || N <= 0 || K <= 0) return cudaSuccess;
+  dim3 grid(K / 128, N / 128, batch);
+  quant_weight_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint4*>(w), N, K, q, scales);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

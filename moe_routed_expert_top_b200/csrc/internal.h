@@ -1,0 +1,62 @@
+// internal.h - launch helpers shared by the C-ABI layer (api.cu) and the
+// kernel translation units. Not part of the public interface.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace moe {
+
+enum GemmMode { kModeStore = 0, kModeSwiglu = 1, kModeSwigluFp8 = 2, kModeFp8Store = 3 };
+
+struct GemmLaunch {
+  int mode = kModeStore;
+  // grouped mode: tables non-null, rows = P; dense mode: tables null, rows = M
+  int rows = 0;
+  int N = 0;  // rows of B per expert
+  int K = 0;
+  int E = 1;
+  const void* A = nullptr;
+  const void* B = nullptr;
+  const float* A_scales = nullptr;  // fp8 mode [rows, K/128]
+  const float* B_scales = nullptr;  // fp8 mode [E, N/128, K/128]
+  const int32_t* group_sizes = nullptr;
+  const int32_t* group_offsets = nullptr;
+  const int32_t* group_padded = nullptr;
+  const int32_t* idx_for_bx = nullptr;
+  int M_blk = 0;  // length of idx_for_bx (grouped mode)
+  void* C = nullptr;
+  float* C_scales = nullptr;
+  float* debug_h = nullptr;
+  int32_t* status = nullptr;
+};
+
+// Each returns cudaSuccess or the launch error.
+cudaError_t launch_grouped_gemm(const GemmLaunch& L, cudaStream_t stream);
+
+cudaError_t launch_route_topk(const float* logits, int T, int E, int k, int score_fn,
+                              int renormalize, int32_t* ids, float* weights, cudaStream_t stream);
+
+cudaError_t launch_tables(const int32_t* ids, int P, int E, int padding_M, int M_blk,
+                          int32_t* sizes, int32_t* offsets, int32_t* padded, int32_t* idx_for_bx,
+                          int32_t* row_of_pair, int32_t* pair_of_row, int32_t* status,
+                          cudaStream_t stream);
+
+cudaError_t launch_gather_rows(const void* hidden, const int32_t* pair_of_row, int P, int k,
+                               int H, void* x_perm, cudaStream_t stream);
+
+cudaError_t launch_unpermute(const void* y, const int32_t* row_of_pair, const float* weights,
+                             int T, int k, int H, float scale, const void* addend, void* out,
+                             cudaStream_t stream);
+
+cudaError_t launch_swiglu_quant(int M, int F, const void* gate_up, const float* h, int out_fp8,
+                                void* out, float* scales, cudaStream_t stream);
+
+cudaError_t launch_quantize_weight(int batch, int N, int K, const void* w, uint8_t* q,
+                                   float* scales, cudaStream_t stream);
+
+// Streaming multiprocessors of the current device (cached per device).
+int device_sm_count();
+
+}  // namespace moe

@@ -373,22 +373,23 @@ def quant_1x128(h32: np.ndarray):
 def quant_weight_128x128(w: np.ndarray):
     """128x128 block FP8 quantisation of a weight matrix w [N, K] (same rule
     as ``quant_1x128`` over each 128x128 block): codes uint8 [N, K] and
-    float32 scales [ceil(N/128), ceil(K/128)]."""
+    float32 scales [ceil(N/128), ceil(K/128)]. N and K are padded with zeros
+    to whole blocks for the block maxima; padding never changes a maximum."""
     w = np.asarray(w, dtype=np.float32)
     N, K = w.shape
     nb, kb = ceil_div(N, 128), ceil_div(K, 128)
-    q = np.zeros((N, K), dtype=np.uint8)
-    s = np.zeros((nb, kb), dtype=np.float32)
-    for i in range(nb):
-        for j in range(kb):
-            blk = w[i * 128:(i + 1) * 128, j * 128:(j + 1) * 128]
-            amax = F32(np.max(np.abs(blk)))
-            if amax > 0:
-                sc = F32(amax / F32(E4M3_MAX))
-                q[i * 128:(i + 1) * 128, j * 128:(j + 1) * 128] = e4m3_encode(
-                    (blk / sc).astype(np.float32))
-                s[i, j] = sc
-    return q, s
+    wp = np.zeros((nb * 128, kb * 128), dtype=np.float32)
+    wp[:N, :K] = w
+    blocks = wp.reshape(nb, 128, kb, 128)
+    amax = np.abs(blocks).max(axis=(1, 3)).astype(np.float32)        # [nb, kb]
+    s = (amax / F32(E4M3_MAX)).astype(np.float32)
+    safe = np.where(amax > 0, s, F32(1.0)).astype(np.float32)
+    scaled = (blocks / safe[:, None, :, None]).astype(np.float32)
+    q = e4m3_encode(scaled)
+    q[np.broadcast_to((amax == 0)[:, None, :, None], q.shape)] = 0
+    q = q.reshape(nb * 128, kb * 128)[:N, :K]
+    s = np.where(amax > 0, s, F32(0.0)).astype(np.float32)
+    return np.ascontiguousarray(q), s
 
 
 _E4M3_VALUES = e4m3_decode_table()

@@ -1,0 +1,128 @@
+"""The C-ABI library loads and exports every entry point include/moe.h declares;
+host-side argument validation and layout logic (no GPU needed: nothing here
+launches a kernel)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_functions():
+    text = open(os.path.join(ROOT, "include", "moe.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def M():
+    from moe_routed_expert_top_b200 import build
+    build.build()
+    import moe_routed_expert_top_b200 as m
+    return m
+
+
+def test_library_exports_every_declared_symbol(M):
+    L = M.lib()
+    declared = _header_functions()
+    assert len(declared) >= 12
+    for name in declared:
+        assert hasattr(L, name), name
+    assert set(declared) == set(M.EXPORTED_SYMBOLS)
+
+
+def test_library_has_no_cuda_driver_load_dependency(M):
+    # loads on a machine without a GPU driver: the runtime is linked statically
+    ctypes.CDLL(M.library_path)
+
+
+def test_status_strings_and_device_status_decoding(M):
+    assert M.moe_status_string(0) == "MOE_OK"
+    assert M.moe_status_string(-3) == "MOE_ERR_WORKSPACE"
+    assert M.moe_decode_device_status(0) == 0
+    assert M.moe_decode_device_status(M.MOE_DEV_TIMEOUT) == -5
+    assert M.moe_decode_device_status(M.MOE_DEV_BAD_EXPERT_ID) == -6
+    assert M.moe_decode_device_status(M.MOE_DEV_TIMEOUT | 1) == -5
+
+
+def test_tables_layout_matches_tutorial_counts(M):
+    p = M.make_problem(T=9, H=128, F=64, E=4, top_k=2, padding_M=128)
+    L = M.moe_get_tables_layout(p)
+    assert L["M_blk"] == 5 and L["P"] == 18
+    offs = [L[k] for k in ("group_sizes", "group_offsets", "group_padded_offsets",
+                           "group_idx_for_bx", "row_of_pair", "pair_of_row")]
+    assert offs == sorted(offs)
+    assert all(o % 4 == 0 for o in offs)        # 16-byte aligned sections
+    assert L["group_offsets"] - L["group_sizes"] >= 4
+    assert L["group_idx_for_bx"] - L["group_padded_offsets"] >= 5
+    assert L["total_int32"] >= L["pair_of_row"] + 18
+
+
+def test_workspace_bytes_covers_intermediates(M):
+    for fp8, Fs in ((False, 0), (True, 0), (False, 2048)):
+        p = M.make_problem(T=512, H=7168, F=2048, E=256, top_k=8, down_fp8=fp8, F_shared=Fs)
+        ws = M.moe_workspace_bytes(p)
+        P = 512 * 8
+        need = P * 7168 * 2 * 2 + P * 2048 * (1 if fp8 else 2)
+        if Fs:
+            need += 512 * Fs * 2 + 512 * 7168 * 2
+        assert ws >= need
+        assert ws % 1024 == 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(E=0), -1), (dict(E=1025), -2), (dict(top_k=33), -2), (dict(top_k=9, E=8), -2),
+    (dict(T=-1), -1), (dict(score_fn=7), -1), (dict(H=100), -2), (dict(padding_M=64), -2),
+    (dict(down_fp8=True, F=192), -2),
+])
+def test_problem_validation(M, kw, status):
+    base = dict(T=16, H=256, F=256, E=8, top_k=2)
+    base.update(kw)
+    p = M.make_problem(**base)
+    # moe_workspace_bytes returns 0 for a problem the forward cannot run
+    assert M.moe_workspace_bytes(p) == 0
+    r = M.lib().moe_experts_forward(ctypes.byref(p), 16, 16, 16, 16, 16, None, None, None,
+                                    ctypes.c_float(1.0), 16, 16, ctypes.c_size_t(1 << 30), None)
+    assert r == status
+
+
+def test_null_pointer_and_workspace_errors(M):
+    p = M.make_problem(T=16, H=256, F=256, E=8, top_k=2)
+    L = M.lib()
+    assert L.moe_route_topk(ctypes.byref(p), None, 16, 16, None) == -1
+    assert L.moe_route_permute(ctypes.byref(p), None, None, None, None, None, 16, 16, None) == -1
+    assert L.moe_unpermute(ctypes.byref(p), None, 16, 16, ctypes.c_float(1.0), None, 16, None) == -1
+    # workspace too small is caught before anything is enqueued
+    assert L.moe_experts_forward(ctypes.byref(p), 16, 16, 16, 16, 16, None, None, None,
+                                 ctypes.c_float(1.0), 16, 16, ctypes.c_size_t(1024), None) == -3
+    # misaligned pointer
+    assert L.moe_experts_forward(ctypes.byref(p), 18, 16, 16, 16, 16, None, None, None,
+                                 ctypes.c_float(1.0), 16, 16, ctypes.c_size_t(1 << 30), None) == -1
+    # FP8 down needs its scales; shared expert needs both weights
+    p8 = M.make_problem(T=16, H=256, F=256, E=8, top_k=2, down_fp8=True)
+    assert L.moe_experts_forward(ctypes.byref(p8), 16, 16, 16, 16, 16, None, None, None,
+                                 ctypes.c_float(1.0), 16, 16, ctypes.c_size_t(1 << 30), None) == -1
+    ps = M.make_problem(T=16, H=256, F=256, E=8, top_k=2, F_shared=128)
+    assert L.moe_experts_forward(ctypes.byref(ps), 16, 16, 16, 16, 16, None, 16, None,
+                                 ctypes.c_float(1.0), 16, 16, ctypes.c_size_t(1 << 30), None) == -1
+    # grouped GEMM: bad epilogue, unsupported K, FP8 with a non-store epilogue
+    assert L.moe_grouped_gemm(None, 128, 256, 256, 16, None, 16, None, None, 9, 16, None, None,
+                              16, None) == -1
+    assert L.moe_grouped_gemm(None, 128, 256, 96, 16, None, 16, None, None, 0, 16, None, None,
+                              16, None) == -2
+    assert L.moe_grouped_gemm(None, 128, 256, 256, 16, 16, 16, 16, None, 1, 16, None, None,
+                              16, None) == -2
+    # swiglu_quant: exactly one of gate_up / h; quantising h needs out_fp8
+    assert L.moe_swiglu_quant(4, 128, None, None, 1, 16, 16, None) == -1
+    assert L.moe_swiglu_quant(4, 128, None, 16, 0, 16, 16, None) == -1
+    assert L.moe_swiglu_quant(4, 126, 16, None, 0, 16, None, None) == -1
+
+
+def test_empty_batch_is_a_no_op(M):
+    p = M.make_problem(T=0, H=256, F=256, E=8, top_k=2)
+    L = M.lib()
+    assert L.moe_route_topk(ctypes.byref(p), None, None, None, None) == 0
+    assert L.moe_experts_forward(ctypes.byref(p), None, None, None, None, None, None, None, None,
+                                 ctypes.c_float(1.0), None, None, ctypes.c_size_t(0), None) == 0

@@ -1,0 +1,161 @@
+"""GPU parity of the whole routed-experts forward (moe_experts_forward)
+against the oracle's per-token definition.
+
+Tolerance |err| <= 1e-2 + 1e-2*|ref| on the bf16 output. The tiny workload and
+mid-size ragged cases are compared on every output element; the four
+production-size workloads on seeded samples of tokens, in the same launch
+configuration the benchmark times. Also: linearity in routed_scaling_factor,
+the dense-MLP reduction, T=1, empty experts, determinism."""
+import numpy as np
+import pytest
+import torch
+
+from moe_inputs import CONFIGS, get_config, make_logits, make_weights
+from oracle import moe_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from tests.gpu_util import ensure_built
+    ensure_built()
+
+
+def _gu():
+    from tests import gpu_util
+    return gpu_util
+
+
+def _run(cfg, hidden, ids, w, weights, scale=None):
+    from moe_routed_expert_top_b200.layer import RoutedExperts
+    layer = RoutedExperts(weights["w_gate_up"], weights["w_down"], cfg.top_k, cfg.score_fn,
+                          cfg.renormalize, cfg.routed_scaling_factor if scale is None else scale,
+                          cfg.down_fp8, weights.get("ws_gate_up"), weights.get("ws_down"))
+    out = layer.forward(hidden, torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda())
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    return out, layer
+
+
+def _oracle(cfg, hidden, ids, w, weights, tokens=None, scale=None, round_output=True):
+    s = cfg.routed_scaling_factor if scale is None else scale
+
+    def loader(name, e):
+        if name in ("w_down_q", "w_down_s"):
+            return None          # the oracle quantises bf16 w_down itself
+        return weights[name][e].float().cpu()
+
+    shared = {}
+    if cfg.F_shared:
+        shared = dict(ws_gate_up=weights["ws_gate_up"].float().cpu(),
+                      ws_down=weights["ws_down"].float().cpu())
+    return O.experts_forward(hidden.float().cpu(), ids, w, None, None, s, tokens=tokens,
+                             fp8=cfg.down_fp8, weight_loader=loader,
+                             round_output=round_output, **shared)
+
+
+def _inputs(cfg, ids=None):
+    gu = _gu()
+    weights = make_weights(cfg, "cuda")
+    g = torch.Generator(device="cuda")
+    g.manual_seed(1000 + cfg.seed)
+    hidden = torch.randn(cfg.T, cfg.H, generator=g, device="cuda").to(torch.bfloat16)
+    if ids is None:
+        ids, w = O.route_topk(make_logits(cfg), cfg.top_k, gu.score_code(cfg), cfg.renormalize)
+    else:
+        _, w = O.route_topk(np.random.default_rng(0).standard_normal((cfg.T, cfg.E)).astype(
+            np.float32), cfg.top_k, gu.score_code(cfg), cfg.renormalize)
+    return hidden, ids, w, weights
+
+
+MID = [
+    get_config("tiny"),
+    get_config("tiny", name="mid_softmax", T=300, E=16, top_k=4, H=256, F=384, seed=21),
+    get_config("tiny", name="mid_sigmoid_shared", T=257, E=12, top_k=3, H=384, F=256,
+               score_fn="sigmoid", routed_scaling_factor=2.5, F_shared=192, seed=22),
+    get_config("tiny", name="mid_fp8", T=190, E=10, top_k=4, H=256, F=512, score_fn="sigmoid",
+               routed_scaling_factor=2.5, down_fp8=True, seed=23),
+]
+
+
+@pytest.mark.parametrize("cfg", MID, ids=[c.name for c in MID])
+def test_forward_all_elements(cfg):
+    gu = _gu()
+    hidden, ids, w, weights = _inputs(cfg)
+    out, _ = _run(cfg, hidden, ids, w, weights)
+    ref = _oracle(cfg, hidden, ids, w, weights)
+    gu.assert_within_tol(gu.f64(out), ref, cfg.name)
+
+
+@pytest.mark.parametrize("name", [n for n in CONFIGS if n != "tiny"])
+def test_forward_full_size_sampled(name):
+    gu = _gu()
+    cfg = get_config(name)
+    hidden, ids, w, weights = _inputs(cfg)
+    out, _ = _run(cfg, hidden, ids, w, weights)
+    rng = np.random.default_rng(7)
+    n = 8 if cfg.H > 4096 else 32
+    # include the tokens routed to the most and the least loaded experts
+    sizes = np.bincount(ids.reshape(-1), minlength=cfg.E)
+    big = int(np.argmax(sizes))
+    small = int(np.argmin(np.where(sizes > 0, sizes, 1 << 30)))
+    t_big = int(np.nonzero((ids == big).any(1))[0][0])
+    t_small = int(np.nonzero((ids == small).any(1))[0][0])
+    tokens = np.unique(np.concatenate([[0, cfg.T - 1, t_big, t_small],
+                                       rng.choice(cfg.T, n, replace=False)]))
+    ref = _oracle(cfg, hidden, ids, w, weights, tokens=tokens)
+    gu.assert_within_tol(gu.f64(out[torch.from_numpy(tokens).cuda()]), ref, name)
+    assert torch.isfinite(out.float()).all()
+
+
+def test_linearity_in_routed_scaling_factor():
+    gu = _gu()
+    cfg = get_config("tiny", name="lin", T=100, E=8, top_k=2, H=256, F=256, seed=31)
+    hidden, ids, w, weights = _inputs(cfg)
+    base, _ = _run(cfg, hidden, ids, w, weights, scale=1.0)
+    ref1 = _oracle(cfg, hidden, ids, w, weights, scale=1.0, round_output=False)
+    for s in (2.5, 2.827):
+        out, _ = _run(cfg, hidden, ids, w, weights, scale=s)
+        gu.assert_within_tol(gu.f64(out), O.bf16_round(s * ref1), f"scale {s}")
+        # each output is one bf16 rounding of s times the same fp32 sum
+        b = gu.f64(base)
+        assert np.all(np.abs(gu.f64(out) - s * b) <= np.abs(s * b) * 2.0 ** -7 + 1e-30)
+
+
+def test_dense_reduction_e1_k1():
+    gu = _gu()
+    cfg = get_config("tiny", name="dense", T=150, E=1, top_k=1, H=256, F=192, seed=32)
+    weights = make_weights(cfg, "cuda")
+    g = torch.Generator(device="cuda")
+    g.manual_seed(3)
+    hidden = torch.randn(cfg.T, cfg.H, generator=g, device="cuda").to(torch.bfloat16)
+    ids = np.zeros((cfg.T, 1), np.int32)
+    w = np.ones((cfg.T, 1), np.float32)
+    out, _ = _run(cfg, hidden, ids, w, weights)
+    ref = O.bf16_round(O.dense_swiglu_mlp(gu.f64(hidden), gu.f64(weights["w_gate_up"][0]),
+                                          gu.f64(weights["w_down"][0])))
+    gu.assert_within_tol(gu.f64(out), ref, "dense reduction")
+
+
+def test_single_token_and_edge_group_sizes():
+    gu = _gu()
+    cfg = get_config("tiny", name="one", T=1, E=8, top_k=2, H=256, F=128, seed=33)
+    hidden, ids, w, weights = _inputs(cfg)
+    out, _ = _run(cfg, hidden, ids, w, weights)
+    gu.assert_within_tol(gu.f64(out), _oracle(cfg, hidden, ids, w, weights), "T=1")
+    sizes = [0, 1, 127, 128, 129, 0, 255, 140]
+    cfg = get_config("tiny", name="edges", T=260, E=8, top_k=3, H=256, F=256, seed=34)
+    ids = gu.random_ids(260, 8, 3, np.random.default_rng(5), sizes=sizes)
+    hidden, ids, w, weights = _inputs(cfg, ids=ids)
+    out, _ = _run(cfg, hidden, ids, w, weights)
+    gu.assert_within_tol(gu.f64(out), _oracle(cfg, hidden, ids, w, weights), "edge sizes")
+
+
+def test_deterministic_repeat():
+    cfg = get_config("tiny", name="det", T=333, E=16, top_k=4, H=256, F=256, seed=35)
+    hidden, ids, w, weights = _inputs(cfg)
+    a, layer = _run(cfg, hidden, ids, w, weights)
+    b = layer.forward(hidden, torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda())
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))

@@ -1,0 +1,265 @@
+"""GPU parity: a4/a6 grouped GEMM (bf16 and FP8 block-scaled), the SwiGLU
+and SwiGLU+FP8 epilogues, the standalone SwiGLU/quant kernel and the 128x128
+weight quantiser, element by element against the oracle.
+
+Shapes span several M-, N- and K-tiles, ragged expert tails, empty experts and
+experts of 1/127/128/129 rows. Tolerance for bf16 outputs: |err| <= 1e-2 +
+1e-2*|ref|. FP8 codes and scales: bit-exact when the oracle quantises the very
+fp32 h the kernel used."""
+import numpy as np
+import pytest
+import torch
+
+from moe_inputs import get_config
+from oracle import moe_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from tests.gpu_util import ensure_built
+    ensure_built()
+
+
+def _gu():
+    from tests import gpu_util
+    return gpu_util
+
+
+def _setup(T, E, k, H, F, seed, sizes=None, std=0.05):
+    """Tables from a routing (oracle-built ids), GPU tables, permuted rows."""
+    gu = _gu()
+    cfg = get_config("tiny", T=T, E=E, top_k=k, H=H, F=F)
+    rng = np.random.default_rng(seed)
+    ids = gu.random_ids(T, E, k, rng, sizes=sizes)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    hidden = torch.randn(T, H, generator=g, device="cuda").to(torch.bfloat16)
+    L, tables, status, x_perm = gu.gpu_tables(cfg, ids, hidden=hidden)
+    ref = O.dispatch_tables(ids, E, 128)
+    wgu = (torch.randn(E, 2 * F, H, generator=g, device="cuda") * std).to(torch.bfloat16)
+    wd = (torch.randn(E, H, F, generator=g, device="cuda") * std).to(torch.bfloat16)
+    return cfg, ids, hidden, L, tables, status, x_perm, ref, wgu, wd
+
+
+def _oracle_rows_gemm(hidden, W, ref, E, k):
+    """Oracle C = A @ B[e]^T over each expert's rows (float64), A = the
+    oracle's own permutation of hidden."""
+    A = O.permute(_gu().f64(hidden), ref["pair_of_row"], k)
+    out = np.zeros((A.shape[0], W.shape[1]))
+    Wf = _gu().f64(W)
+    for e in range(E):
+        a, b = ref["group_offsets"][e], ref["group_offsets"][e + 1]
+        if b > a:
+            out[a:b] = O.gate_up_rows(A[a:b], Wf[e])
+    return out
+
+
+GEMM_CASES = [
+    # T, E, k, H, F, sizes
+    (9, 4, 2, 128, 64, None),
+    (200, 8, 2, 256, 384, None),
+    (260, 8, 3, 512, 128, [0, 1, 127, 128, 129, 0, 255, 140]),
+    (300, 5, 1, 192, 256, [0, 0, 300, 0, 0]),
+]
+
+
+@pytest.mark.parametrize("T,E,k,H,F,sizes", GEMM_CASES)
+def test_grouped_gemm_store(T, E, k, H, F, sizes):
+    gu = _gu()
+    import moe_routed_expert_top_b200 as M
+    cfg, ids, hidden, L, tables, status, x_perm, ref, wgu, wd = _setup(T, E, k, H, F, 1, sizes)
+    prob = gu.problem(cfg)
+    C = torch.full((L["P"], 2 * F), float("nan"), dtype=torch.bfloat16, device="cuda")
+    M.moe_grouped_gemm(prob, 0, 2 * F, H, x_perm, None, wgu, None, tables, M.MOE_EPI_STORE, C,
+                       None, None, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    gu.assert_within_tol(gu.f64(C), _oracle_rows_gemm(hidden, wgu, ref, E, k), "gate_up store")
+
+
+@pytest.mark.parametrize("T,E,k,H,F,sizes", GEMM_CASES)
+def test_grouped_gemm_swiglu(T, E, k, H, F, sizes):
+    gu = _gu()
+    import moe_routed_expert_top_b200 as M
+    cfg, ids, hidden, L, tables, status, x_perm, ref, wgu, wd = _setup(T, E, k, H, F, 2, sizes)
+    prob = gu.problem(cfg)
+    h = torch.full((L["P"], F), float("nan"), dtype=torch.bfloat16, device="cuda")
+    M.moe_grouped_gemm(prob, 0, 2 * F, H, x_perm, None, wgu, None, tables, M.MOE_EPI_SWIGLU, h,
+                       None, None, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    G = _oracle_rows_gemm(hidden, wgu, ref, E, k)
+    gu.assert_within_tol(gu.f64(h), O.bf16_round(O.swiglu(G, F)), "swiglu epilogue")
+
+
+@pytest.mark.parametrize("T,E,k,H,F,sizes", [c for c in GEMM_CASES if c[4] % 128 == 0])
+def test_grouped_gemm_swiglu_fp8_epilogue(T, E, k, H, F, sizes):
+    gu = _gu()
+    import moe_routed_expert_top_b200 as M
+    cfg, ids, hidden, L, tables, status, x_perm, ref, wgu, wd = _setup(T, E, k, H, F, 3, sizes)
+    prob = gu.problem(cfg)
+    P = L["P"]
+    q = torch.zeros(P, F, dtype=torch.uint8, device="cuda")
+    s = torch.zeros(P, F // 128, dtype=torch.float32, device="cuda")
+    dh = torch.zeros(P, F, dtype=torch.float32, device="cuda")
+    M.moe_grouped_gemm(prob, 0, 2 * F, H, x_perm, None, wgu, None, tables, M.MOE_EPI_SWIGLU_FP8,
+                       q, s, dh, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    # against the oracle: the fused fp32 h, the scales and the dequantised codes
+    G = _oracle_rows_gemm(hidden, wgu, ref, E, k)
+    h_ref = O.swiglu(G, F)
+    h32 = dh.cpu().numpy().astype(np.float64)
+    gu.assert_within_tol(h32, h_ref, "fused h", rtol=1e-3, atol=1e-4)
+    amax = np.abs(h_ref).reshape(P, F // 128, 128).max(2)
+    gu.assert_within_tol(s.cpu().numpy(), amax / 448, "scales", rtol=1e-3, atol=1e-7)
+    deq = O.e4m3_value(q.cpu().numpy()) * np.repeat(s.cpu().numpy().astype(np.float64), 128, 1)
+    bound = np.abs(h_ref) * (2.0 ** -4 + 2e-3) + np.repeat(amax / 448, 128, 1) * (2.0 ** -9 + 1e-3)
+    assert np.all(np.abs(deq - h_ref) <= bound)
+    # the fused epilogue and the standalone quantiser agree byte for byte on the
+    # same fp32 h (the standalone one is bit-exact against the oracle)
+    q2 = torch.zeros_like(q)
+    s2 = torch.zeros_like(s)
+    M.moe_swiglu_quant(P, F, None, dh, 1, q2, s2)
+    torch.cuda.synchronize()
+    assert torch.equal(q2, q) and torch.equal(s2.view(torch.int32), s.view(torch.int32))
+
+
+@pytest.mark.parametrize("T,E,k,H,F,sizes", [(200, 8, 2, 256, 384, None),
+                                            (260, 8, 3, 512, 256, [0, 1, 127, 128, 129, 0, 255, 140])])
+def test_grouped_gemm_fp8_block_scaled(T, E, k, H, F, sizes):
+    gu = _gu()
+    import moe_routed_expert_top_b200 as M
+    cfg, ids, hidden, L, tables, status, x_perm, ref, wgu, wd = _setup(T, E, k, H, F, 4, sizes)
+    prob = gu.problem(cfg)
+    P = L["P"]
+    # activations: oracle-quantised random h (so both sides see the same codes)
+    rng = np.random.default_rng(9)
+    h = (rng.standard_normal((P, F)) * rng.uniform(0.1, 3, (P, 1))).astype(np.float32)
+    qa, sa = O.quant_1x128(h)
+    wq, ws = zip(*[O.quant_weight_128x128(gu.f64(wd[e]).astype(np.float32)) for e in range(E)])
+    wq, ws = np.stack(wq), np.stack(ws)
+    y = torch.full((P, H), float("nan"), dtype=torch.bfloat16, device="cuda")
+    M.moe_grouped_gemm(prob, 0, H, F, torch.from_numpy(qa).cuda(), torch.from_numpy(sa).cuda(),
+                       torch.from_numpy(wq).cuda(), torch.from_numpy(ws).cuda(), tables,
+                       M.MOE_EPI_STORE, y, None, None, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    refy = np.zeros((P, H))
+    for e in range(E):
+        a, b = ref["group_offsets"][e], ref["group_offsets"][e + 1]
+        if b > a:
+            refy[a:b] = O.fp8_block_scaled_matmul(qa[a:b], sa[a:b], wq[e], ws[e])
+    gu.assert_within_tol(gu.f64(y), refy, "fp8 down")
+
+
+@pytest.mark.parametrize("M_rows,N,K", [(1, 128, 64), (300, 512, 448), (4096 + 17, 256, 256)])
+def test_dense_gemm_store(M_rows, N, K):
+    gu = _gu()
+    import moe_routed_expert_top_b200 as M
+    g = torch.Generator(device="cuda")
+    g.manual_seed(M_rows)
+    A = torch.randn(M_rows, K, generator=g, device="cuda").to(torch.bfloat16)
+    B = (torch.randn(N, K, generator=g, device="cuda") * 0.05).to(torch.bfloat16)
+    C = torch.empty(M_rows, N, dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    M.moe_grouped_gemm(None, M_rows, N, K, A, None, B, None, None, M.MOE_EPI_STORE, C, None, None,
+                       status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    gu.assert_within_tol(gu.f64(C), gu.f64(A) @ gu.f64(B).T, "dense")
+
+
+@pytest.mark.parametrize("Mr,F", [(0, 128), (1, 6144), (127, 6144), (128, 6144), (129, 6144),
+                                  (37, 200)])
+def test_swiglu_quant_from_h_bit_exact(Mr, F):
+    import moe_routed_expert_top_b200 as M
+    rng = np.random.default_rng(Mr + F)
+    h = (rng.standard_normal((Mr, F)) * rng.uniform(1e-3, 30, (Mr, 1))).astype(np.float32)
+    if Mr > 3:
+        h[1, :128] = 0.0
+        h[2, 5] = -1e-30
+        h[3, :] *= 1e-4
+    q = torch.zeros(Mr, F, dtype=torch.uint8, device="cuda")
+    s = torch.zeros(Mr, -(-F // 128), dtype=torch.float32, device="cuda")
+    M.moe_swiglu_quant(Mr, F, None, torch.from_numpy(h).cuda() if Mr else None, 1, q, s)
+    torch.cuda.synchronize()
+    rq, rs = O.quant_1x128(h)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+    assert np.array_equal(q.cpu().numpy(), rq)
+
+
+def test_e4m3_encoder_sweep_through_quant():
+    """Rows whose amax is exactly 448 have scale 1, so the kernel's codes are
+    the E4M3 encoding of h itself: sweep dense values in [-448, 448]."""
+    import moe_routed_expert_top_b200 as M
+    rng = np.random.default_rng(0)
+    n = 1 << 22
+    mags = np.exp(rng.uniform(np.log(2.0 ** -12), np.log(448.0), n))
+    vals = (mags * rng.choice([-1.0, 1.0], n)).astype(np.float32)
+    v = O.e4m3_decode_table()
+    finite = v[np.isfinite(v)]
+    mids = ((np.sort(finite)[1:] + np.sort(finite)[:-1]) / 2).astype(np.float32)
+    vals = np.concatenate([vals, mids, finite.astype(np.float32), -mids,
+                           np.array([-0.0, 0.0, 2.0 ** -11, -(2.0 ** -11)], np.float32)])
+    vals = np.clip(vals, -448, 448)
+    cols = 128
+    rows = -(-vals.size // (cols - 1))
+    h = np.zeros((rows, cols), np.float32)
+    flat = np.zeros(rows * (cols - 1), np.float32)
+    flat[:vals.size] = vals
+    h[:, 1:] = flat.reshape(rows, cols - 1)
+    h[:, 0] = 448.0
+    q = torch.zeros(rows, cols, dtype=torch.uint8, device="cuda")
+    s = torch.zeros(rows, 1, dtype=torch.float32, device="cuda")
+    M.moe_swiglu_quant(rows, cols, None, torch.from_numpy(h).cuda(), 1, q, s)
+    torch.cuda.synchronize()
+    assert np.all(s.cpu().numpy() == 1.0)
+    assert np.array_equal(q.cpu().numpy(), O.e4m3_encode(h))
+
+
+@pytest.mark.parametrize("out_fp8", [0, 1])
+def test_swiglu_quant_from_gate_up(out_fp8):
+    gu = _gu()
+    import moe_routed_expert_top_b200 as M
+    Mr, F = 257, 384
+    g = torch.Generator(device="cuda")
+    g.manual_seed(3)
+    gate_up = (torch.randn(Mr, 2 * F, generator=g, device="cuda") * 2).to(torch.bfloat16)
+    h_ref = O.swiglu(gu.f64(gate_up), F)
+    if out_fp8:
+        q = torch.zeros(Mr, F, dtype=torch.uint8, device="cuda")
+        s = torch.zeros(Mr, F // 128, dtype=torch.float32, device="cuda")
+        M.moe_swiglu_quant(Mr, F, gate_up, None, 1, q, s)
+        torch.cuda.synchronize()
+        deq = O.e4m3_value(q.cpu().numpy()) * np.repeat(s.cpu().numpy().astype(np.float64), 128, 1)
+        amax = np.abs(h_ref).reshape(Mr, F // 128, 128).max(2)
+        assert np.allclose(s.cpu().numpy(), amax / 448, rtol=1e-5)
+        # E4M3 keeps 3 mantissa bits: half-ulp relative error 2**-4 (plus subnormals)
+        err = np.abs(deq - h_ref)
+        assert np.all(err <= np.abs(h_ref) * (2.0 ** -4 + 1e-5) + np.repeat(amax / 448, 128, 1) * 2.0 ** -9)
+    else:
+        out = torch.empty(Mr, F, dtype=torch.bfloat16, device="cuda")
+        M.moe_swiglu_quant(Mr, F, gate_up, None, 0, out, None)
+        torch.cuda.synchronize()
+        gu.assert_within_tol(gu.f64(out), O.bf16_round(h_ref), "swiglu bf16", rtol=1e-2, atol=1e-3)
+
+
+def test_weight_quant_bit_exact():
+    gu = _gu()
+    import moe_routed_expert_top_b200 as M
+    E, N, K = 3, 384, 256
+    g = torch.Generator(device="cuda")
+    g.manual_seed(8)
+    w = (torch.randn(E, N, K, generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+    w[1, 128:256, 128:] = 0
+    q = torch.zeros(E, N, K, dtype=torch.uint8, device="cuda")
+    s = torch.zeros(E, N // 128, K // 128, dtype=torch.float32, device="cuda")
+    M.moe_quantize_weight_128x128(E, N, K, w, q, s)
+    torch.cuda.synchronize()
+    for e in range(E):
+        rq, rs = O.quant_weight_128x128(gu.f64(w[e]).astype(np.float32))
+        assert np.array_equal(q[e].cpu().numpy(), rq)
+        assert np.array_equal(s[e].cpu().numpy().view(np.uint32), rs.view(np.uint32))
