@@ -26,13 +26,11 @@ written from these pages:
 
 Precision: every sum and product the pages leave open runs in float64. Where a
 floating-point value decides an integer (the FP8 code, the top-k order) the
-oracle takes that decision in float32, the precision the kernels use. The
-tensors the pages' pipeline hands from one kernel to the next are bf16, and the
-oracle rounds them the same way (exact round-to-nearest-even from float64): h,
-the down GEMM's operand; y, each grouped GEMM output row (PR #1580's grouped
-GEMM returns bf16 C and its unpermute scales before the final cast); the shared
-expert's output (PR #778 adds shared_out to routed_out as tensors); and the
-final output.
+oracle takes that decision in float32, the precision the kernels use. Two bf16
+roundings belong to the method itself and are done here as exact
+round-to-nearest-even from float64: h, because the down GEMM multiplies bf16
+(or E4M3) operands, and the final bf16 output. The down GEMM's result y and the
+shared expert's output are sums, kept in float64 up to the final cast.
 
 Parity status per function (what pins it is in ``tests/test_oracle_*.py``):
 every function below is pinned except ``experts_forward`` end-to-end values,
@@ -509,8 +507,7 @@ def experts_forward(hidden, topk_ids_, topk_weights, w_gate_up, w_down, scale: f
                     tokens=None, fp8: bool = False, w_down_q=None, w_down_s=None,
                     ws_gate_up=None, ws_down=None, weight_loader=None,
                     round_output: bool = True):
-    """out[t] = bf16( scale * sum_j w[t,j] * bf16(MLP_{e(t,j)}(hidden[t]))
-                      + bf16(shared(hidden[t])) )
+    """out[t] = bf16( scale * sum_j w[t,j] * MLP_{e(t,j)}(hidden[t]) + shared(hidden[t]) )
 
     Computed straight from the definition, per (token, expert) pair, with no
     permutation: pairs are grouped by expert only so each expert's weights are
@@ -534,15 +531,15 @@ def experts_forward(hidden, topk_ids_, topk_weights, w_gate_up, w_down, scale: f
         return None if src is None else src[e]
 
     sub_ids = ids[toks]
-    Y = np.zeros((len(toks), k, H), dtype=np.float64)   # bf16 MLP output of every pair
+    Y = np.zeros((len(toks), k, H), dtype=np.float64)   # MLP output of every pair
     for e in np.unique(sub_ids):
         ti, ji = np.nonzero(sub_ids == e)
-        Y[ti, ji] = bf16_round(expert_mlp(X[ti], load("w_gate_up", e), load("w_down", e), fp8=fp8,
+        Y[ti, ji] = expert_mlp(X[ti], load("w_gate_up", e), load("w_down", e), fp8=fp8,
                                w_down_q_e=load("w_down_q", e) if fp8 else None,
-                               w_down_s_e=load("w_down_s", e) if fp8 else None))
+                               w_down_s_e=load("w_down_s", e) if fp8 else None)
     for j in range(k):                                   # slot order
         acc += w[toks, j][:, None] * Y[:, j]
     acc = float(scale) * acc
     if ws_gate_up is not None:
-        acc = acc + bf16_round(dense_swiglu_mlp(X, ws_gate_up, ws_down))
+        acc = acc + dense_swiglu_mlp(X, ws_gate_up, ws_down)
     return bf16_round(acc) if round_output else acc

@@ -83,7 +83,7 @@ def test_dense_reduction_to_textbook_swiglu_mlp():
     out = O.experts_forward(x, ids, w, wgu, wd, 1.0, round_output=False)
     xs, g, d = x.float().numpy(), wgu[0].float().numpy(), wd[0].float().numpy()
     for t in range(T):
-        ref = O.bf16_round(_textbook_mlp_token(xs[t], g, d, F))   # bf16 GEMM output y
+        ref = _textbook_mlp_token(xs[t], g, d, F)
         assert np.allclose(out[t], ref, rtol=1e-12, atol=1e-12)
 
 
@@ -102,8 +102,7 @@ def test_brute_force_tiny_moe():
         ref = [0.0] * H
         for j in range(k):
             e = int(ids[t, j])
-            y = O.bf16_round(_textbook_mlp_token(xs[t], wgu[e].float().numpy(),
-                                                 wd[e].float().numpy(), F))
+            y = _textbook_mlp_token(xs[t], wgu[e].float().numpy(), wd[e].float().numpy(), F)
             for n in range(H):
                 ref[n] += float(w[t, j]) * y[n]
         ref = [s * v for v in ref]
@@ -129,7 +128,7 @@ def test_table_pipeline_equals_per_token_definition(fp8):
     for bx in range(t["M_blk"]):
         g, m0, rows = O.block_rows(t, bx, bt)
         if rows:
-            y[m0:m0 + rows] = O.bf16_round(O.expert_mlp(xp[m0:m0 + rows], wgu[g], wd[g], fp8=fp8))
+            y[m0:m0 + rows] = O.expert_mlp(xp[m0:m0 + rows], wgu[g], wd[g], fp8=fp8)
     out = O.unpermute(y, t["row_of_pair"], w, s, round_output=False)
     assert np.allclose(out, ref, rtol=1e-12, atol=1e-12)
     # the sampled-token form gives the same rows
