@@ -73,7 +73,7 @@ def work_model(cfg, ids: np.ndarray) -> dict:
     total_bytes = w_gu + w_dn + w_sh + act
     # gate+up kernel alone: its weights, its A rows (x_perm), its h output
     gu_bytes = w_gu + P * H * 2 + P * F * (1 if cfg.down_fp8 else 2) + (P * (F // 128) * 4 if cfg.down_fp8 else 0)
-    dn_bytes = w_dn + P * F * (1 if cfg.down_fp8 else 2) + P * H * 2
+    dn_bytes = w_dn + P * F * (1 if cfg.down_fp8 else 2) + P * H * 4
     return dict(touched=touched, flops=flops_routed + flops_shared, flops_routed=flops_routed,
                 bytes=total_bytes, gate_up_bytes=gu_bytes, gate_up_flops=4.0 * P * H * F,
                 down_bytes=dn_bytes, down_flops=2.0 * P * H * F)
@@ -194,12 +194,12 @@ def stage_breakdown(M, layer, cfg, hidden, ids, weights, steps, flush):
     else:
         h = torch.empty(P, cfg.F, dtype=torch.bfloat16, device=dev)
         hs = None
-    y = torch.empty(P, cfg.H, dtype=torch.bfloat16, device=dev)
+    y = torch.empty(P, cfg.H, dtype=torch.float32, device=dev)
     out = torch.empty(T, cfg.H, dtype=torch.bfloat16, device=dev)
     addend = None
     if cfg.F_shared:
         sh = torch.empty(T, cfg.F_shared, dtype=torch.bfloat16, device=dev)
-        addend = torch.empty(T, cfg.H, dtype=torch.bfloat16, device=dev)
+        addend = torch.empty(T, cfg.H, dtype=torch.float32, device=dev)
     del ws
     stages = {
         "route_permute": lambda: M.moe_route_permute(prob, None, ids, None, hidden, x_perm,
@@ -209,15 +209,15 @@ def stage_breakdown(M, layer, cfg, hidden, ids, weights, steps, flush):
             M.MOE_EPI_SWIGLU_FP8 if cfg.down_fp8 else M.MOE_EPI_SWIGLU, h, hs, None, status),
         "down_gemm": lambda: M.moe_grouped_gemm(
             prob, 0, cfg.H, cfg.F, h, hs, layer.w_down, layer.w_down_scales, tables,
-            M.MOE_EPI_STORE, y, None, None, status),
+            M.MOE_EPI_STORE_F32, y, None, None, status),
     }
     if cfg.F_shared:
         stages["shared_gate_up_gemm"] = lambda: M.moe_grouped_gemm(
             None, T, 2 * cfg.F_shared, cfg.H, hidden, None, layer.ws_gate_up, None, None,
             M.MOE_EPI_SWIGLU, sh, None, None, status)
         stages["shared_down_gemm"] = lambda: M.moe_grouped_gemm(
-            None, T, cfg.H, cfg.F_shared, sh, None, layer.ws_down, None, None, M.MOE_EPI_STORE,
-            addend, None, None, status)
+            None, T, cfg.H, cfg.F_shared, sh, None, layer.ws_down, None, None,
+            M.MOE_EPI_STORE_F32, addend, None, None, status)
     stages["unpermute"] = lambda: M.moe_unpermute(prob, y, tables, weights,
                                                   cfg.routed_scaling_factor, addend, out)
     stream = torch.cuda.current_stream()

@@ -91,7 +91,8 @@ enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 };
 enum {
   MOE_EPI_STORE = 0,       /* C bf16 [rows, N] = A @ B^T */
   MOE_EPI_SWIGLU = 1,      /* C bf16 [rows, N/2] = SiLU(G[:, :N/2]) * G[:, N/2:] */
-  MOE_EPI_SWIGLU_FP8 = 2   /* C e4m3 [rows, N/2] + C_scales fp32 [rows, N/256] */
+  MOE_EPI_SWIGLU_FP8 = 2,  /* C e4m3 [rows, N/2] + C_scales fp32 [rows, N/256] */
+  MOE_EPI_STORE_F32 = 3    /* C fp32 [rows, N] = A @ B^T (the accumulator, unrounded) */
 };
 
 /* One MoE layer's shape and routing options. */
@@ -175,6 +176,7 @@ moe_status moe_route_permute(const moe_problem* prob, const float* logits,
  *   tables null (dense, one group): A [M_rows, K], B [N, K].
  * bf16 mode (A_scales == B_scales == NULL): A, B bf16; K % 64 == 0.
  *   MOE_EPI_STORE:      C bf16 [rows, N], N % 64 == 0.
+ *   MOE_EPI_STORE_F32:  C fp32 [rows, N], N % 64 == 0.
  *   MOE_EPI_SWIGLU:     N = 2F with gate = B rows [0,F), up = rows [F,2F)
  *                       ([PR778] Design); C bf16 [rows, F]; F % 64 == 0.
  *   MOE_EPI_SWIGLU_FP8: as SWIGLU, then per row and 128-column tile
@@ -184,8 +186,9 @@ moe_status moe_route_permute(const moe_problem* prob, const float* logits,
  *                       debug_h (nullable) receives the fp32 h [rows, F].
  * FP8 mode (A_scales and B_scales non-null): A e4m3 [rows, K] with A_scales
  *   fp32 [rows, K/128]; B e4m3 [E, N, K] with B_scales fp32 [E, N/128, K/128];
- *   C bf16 [rows, N] = sum over K-blocks kb of sa[r,kb]*sb[n/128,kb]*(A_kb @ B_kb^T);
- *   epilogue must be MOE_EPI_STORE; N % 128 == 0, K % 128 == 0.
+ *   C [rows, N] = sum over K-blocks kb of sa[r,kb]*sb[n/128,kb]*(A_kb @ B_kb^T),
+ *   bf16 with MOE_EPI_STORE or fp32 with MOE_EPI_STORE_F32; N % 128 == 0,
+ *   K % 128 == 0.
  * Device flags: MOE_DEV_TIMEOUT into *dev_status (required). */
 moe_status moe_grouped_gemm(const moe_problem* prob, int32_t M_rows, int32_t N, int32_t K,
                             const void* A, const float* A_scales,
@@ -206,10 +209,12 @@ moe_status moe_swiglu_quant(int32_t M, int32_t F, const void* gate_up, const flo
 
 /* a7 ([PR1580] Unpermute): out bf16 [T, H] =
  *   RNE_bf16( scale * sum_{j<k} topk_weights[t,j] * y[row_of_pair[t*k+j]] + addend[t] )
- * with the sum in fp32 in slot order j; y bf16 [P, H]; addend bf16 [T, H] or
- * NULL; tables as written by moe_route_permute (row -1 contributes nothing). */
-moe_status moe_unpermute(const moe_problem* prob, const void* y, const int32_t* tables,
-                         const float* topk_weights, float scale, const void* addend,
+ * with the sum in fp32 in slot order j; y fp32 [P, H] (the down GEMM's
+ * MOE_EPI_STORE_F32 output: kept unrounded so a bf16 intermediate adds no
+ * error before the single final cast); addend fp32 [T, H] or NULL; tables as
+ * written by moe_route_permute (row -1 contributes nothing). */
+moe_status moe_unpermute(const moe_problem* prob, const float* y, const int32_t* tables,
+                         const float* topk_weights, float scale, const float* addend,
                          void* out, moe_stream_t stream);
 
 /* Offline weight preparation for the FP8 down GEMM: for each of `batch`

@@ -19,7 +19,7 @@ __all__ = [
     "moe_grouped_gemm", "moe_swiglu_quant", "moe_unpermute", "moe_quantize_weight_128x128",
     "moe_experts_forward", "moe_decode_device_status", "moe_status_string",
     "moe_last_launch_count", "EXPORTED_SYMBOLS",
-    "MOE_OK", "MOE_EPI_STORE", "MOE_EPI_SWIGLU", "MOE_EPI_SWIGLU_FP8",
+    "MOE_OK", "MOE_EPI_STORE", "MOE_EPI_SWIGLU", "MOE_EPI_SWIGLU_FP8", "MOE_EPI_STORE_F32",
     "MOE_SCORE_SOFTMAX", "MOE_SCORE_SIGMOID", "MOE_DEV_BAD_EXPERT_ID", "MOE_DEV_TIMEOUT",
 ]
 
@@ -31,7 +31,7 @@ MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE = -1, -2, -3
 MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_DEVICE_FLAG = -4, -5, -6
 MOE_DEV_BAD_EXPERT_ID, MOE_DEV_TIMEOUT, MOE_DEV_BAD_TABLES = 1, 2, 4
 MOE_SCORE_SOFTMAX, MOE_SCORE_SIGMOID = 0, 1
-MOE_EPI_STORE, MOE_EPI_SWIGLU, MOE_EPI_SWIGLU_FP8 = 0, 1, 2
+MOE_EPI_STORE, MOE_EPI_SWIGLU, MOE_EPI_SWIGLU_FP8, MOE_EPI_STORE_F32 = 0, 1, 2, 3
 
 EXPORTED_SYMBOLS = (
     "moe_get_tables_layout", "moe_workspace_bytes", "moe_route_topk", "moe_route_permute",

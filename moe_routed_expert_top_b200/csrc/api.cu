@@ -94,9 +94,9 @@ WorkspacePlan plan_workspace(const moe_problem* pr) {
   w.x_perm = take(P * H * 2);
   w.h = take(P * F * (pr->down_fp8 ? 1 : 2));
   w.h_scales = take(pr->down_fp8 ? P * (F / 128) * 4 : 0);
-  w.y = take(P * H * 2);
+  w.y = take(P * H * 4);               // fp32: the down GEMM's accumulator, unrounded
   w.hs = take(Fs ? T * Fs * 2 : 0);
-  w.ys = take(Fs ? T * H * 2 : 0);
+  w.ys = take(Fs ? T * H * 4 : 0);
   w.total = o;
   return w;
 }
@@ -191,15 +191,18 @@ moe_status moe_grouped_gemm(const moe_problem* prob, int32_t M_rows, int32_t N, 
   }
   if (g.rows == 0) return MOE_OK;
   if (fp8) {
-    if (epilogue != MOE_EPI_STORE) return MOE_ERR_UNSUPPORTED;
+    if (epilogue != MOE_EPI_STORE && epilogue != MOE_EPI_STORE_F32) return MOE_ERR_UNSUPPORTED;
     if (N % 128 != 0 || K % 128 != 0) return MOE_ERR_UNSUPPORTED;
     g.mode = moe::kModeFp8Store;
+    g.out_f32 = epilogue == MOE_EPI_STORE_F32;
   } else {
     if (K % 64 != 0) return MOE_ERR_UNSUPPORTED;
     switch (epilogue) {
       case MOE_EPI_STORE:
+      case MOE_EPI_STORE_F32:
         if (N % 64 != 0) return MOE_ERR_UNSUPPORTED;
         g.mode = moe::kModeStore;
+        g.out_f32 = epilogue == MOE_EPI_STORE_F32;
         break;
       case MOE_EPI_SWIGLU:
         if (N % 128 != 0) return MOE_ERR_UNSUPPORTED;  // F = N/2 multiple of 64
@@ -244,8 +247,8 @@ moe_status moe_swiglu_quant(int32_t M, int32_t F, const void* gate_up, const flo
   return MOE_OK;
 }
 
-moe_status moe_unpermute(const moe_problem* prob, const void* y, const int32_t* tables,
-                         const float* topk_weights, float scale, const void* addend, void* out,
+moe_status moe_unpermute(const moe_problem* prob, const float* y, const int32_t* tables,
+                         const float* topk_weights, float scale, const float* addend, void* out,
                          moe_stream_t stream) {
   moe_status s = check_problem(prob, false);
   if (s != MOE_OK) return s;
@@ -304,7 +307,7 @@ moe_status moe_experts_forward(const moe_problem* prob, const void* hidden,
   void* x_perm = base + w.x_perm;
   void* h = base + w.h;
   float* h_scales = reinterpret_cast<float*>(base + w.h_scales);
-  void* y = base + w.y;
+  float* y = reinterpret_cast<float*>(base + w.y);
   moe_tables_layout L;
   fill_layout(prob, &L);
   const int T = prob->T, H = prob->H, F = prob->F, E = prob->E, k = prob->top_k;
@@ -345,12 +348,13 @@ moe_status moe_experts_forward(const moe_problem* prob, const void* hidden,
   g.A_scales = prob->down_fp8 ? h_scales : nullptr;
   g.B_scales = prob->down_fp8 ? w_down_scales : nullptr;
   g.C = y;
+  g.out_f32 = 1;
   g.C_scales = nullptr;
   MOE_CUDA_TRY(moe::launch_grouped_gemm(g, st));
   g_last_launches += 2;
 
   // shared expert: a dense SwiGLU MLP on all tokens, added in the unpermute
-  const void* addend = nullptr;
+  const float* addend = nullptr;
   if (prob->F_shared > 0) {
     moe::GemmLaunch d;
     d.rows = T;
@@ -369,8 +373,9 @@ moe_status moe_experts_forward(const moe_problem* prob, const void* hidden,
     d.A = base + w.hs;
     d.B = ws_down;
     d.C = base + w.ys;
+    d.out_f32 = 1;
     MOE_CUDA_TRY(moe::launch_grouped_gemm(d, st));
-    addend = base + w.ys;
+    addend = reinterpret_cast<const float*>(base + w.ys);
     g_last_launches += 2;
   }
   // a7

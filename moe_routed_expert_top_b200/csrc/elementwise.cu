@@ -14,17 +14,18 @@ namespace moe {
 // ---------------------------------------------------------------------------
 // a7: out[t] = bf16( scale * sum_j w[t,j] * y[row_of_pair[t*k+j]] + addend[t] )
 // (TileOPs PR #1580, Unpermute: scaling folded in before the cast/store; the
-// result is written straight into the caller's output buffer). One thread per
-// 8 columns of one token; fp32 accumulation in slot order j.
+// result is written straight into the caller's output buffer). y and the
+// addend are fp32 (the down GEMM's accumulator, not rounded in between). One
+// thread per 8 columns of one token; fp32 accumulation in slot order j.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) unpermute_kernel(const uint4* __restrict__ y,
+__global__ void __launch_bounds__(128) unpermute_kernel(const float4* __restrict__ y,
                                                         const int32_t* __restrict__ row_of_pair,
                                                         const float* __restrict__ w, int k,
                                                         int P, int H8, float scale,
-                                                        const uint4* __restrict__ addend,
+                                                        const float4* __restrict__ addend,
                                                         uint4* __restrict__ out) {
   const int t = blockIdx.y;
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;  // 8-column group
   if (c >= H8) return;
   float acc[8];
 #pragma unroll
@@ -34,37 +35,41 @@ __global__ void __launch_bounds__(128) unpermute_kernel(const uint4* __restrict_
     const int row = __ldg(row_of_pair + pbase + j);
     if (row < 0 || row >= P) continue;
     const float wt = __ldg(w + pbase + j);
-    const uint4 v = __ldg(y + static_cast<int64_t>(row) * H8 + c);
-    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      acc[2 * i] = fmaf(wt, bf16lo_to_f32(u[i]), acc[2 * i]);
-      acc[2 * i + 1] = fmaf(wt, bf16hi_to_f32(u[i]), acc[2 * i + 1]);
-    }
+    const float4* src = y + (static_cast<int64_t>(row) * H8 + c) * 2;
+    const float4 a = __ldg(src), b = __ldg(src + 1);
+    acc[0] = fmaf(wt, a.x, acc[0]);
+    acc[1] = fmaf(wt, a.y, acc[1]);
+    acc[2] = fmaf(wt, a.z, acc[2]);
+    acc[3] = fmaf(wt, a.w, acc[3]);
+    acc[4] = fmaf(wt, b.x, acc[4]);
+    acc[5] = fmaf(wt, b.y, acc[5]);
+    acc[6] = fmaf(wt, b.z, acc[6]);
+    acc[7] = fmaf(wt, b.w, acc[7]);
   }
-  uint32_t o[4];
+  float v[8];
   if (addend != nullptr) {
-    const uint4 a = __ldg(addend + static_cast<int64_t>(t) * H8 + c);
-    const uint32_t au[4] = {a.x, a.y, a.z, a.w};
+    const float4* ad = addend + (static_cast<int64_t>(t) * H8 + c) * 2;
+    const float4 a = __ldg(ad), b = __ldg(ad + 1);
+    const float add[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      o[i] = pack_bf16x2(fmaf(scale, acc[2 * i], bf16lo_to_f32(au[i])),
-                         fmaf(scale, acc[2 * i + 1], bf16hi_to_f32(au[i])));
+    for (int i = 0; i < 8; ++i) v[i] = fmaf(scale, acc[i], add[i]);
   } else {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) o[i] = pack_bf16x2(scale * acc[2 * i], scale * acc[2 * i + 1]);
+    for (int i = 0; i < 8; ++i) v[i] = scale * acc[i];
   }
-  out[static_cast<int64_t>(t) * H8 + c] = make_uint4(o[0], o[1], o[2], o[3]);
+  out[static_cast<int64_t>(t) * H8 + c] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                                     pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
 }
 
-cudaError_t launch_unpermute(const void* y, const int32_t* row_of_pair, const float* weights,
-                             int T, int k, int H, float scale, const void* addend, void* out,
+cudaError_t launch_unpermute(const float* y, const int32_t* row_of_pair, const float* weights,
+                             int T, int k, int H, float scale, const float* addend, void* out,
                              cudaStream_t stream) {
   if (T <= 0) return cudaSuccess;
   const int H8 = H / 8;
   dim3 grid((H8 + 127) / 128, T);
-  unpermute_kernel<<<grid, 128, 0, stream>>>(static_cast<const uint4*>(y), row_of_pair, weights, k,
-                                             T * k, H8, scale, static_cast<const uint4*>(addend),
+  unpermute_kernel<<<grid, 128, 0, stream>>>(reinterpret_cast<const float4*>(y), row_of_pair,
+                                             weights, k, T * k, H8, scale,
+                                             reinterpret_cast<const float4*>(addend),
                                              static_cast<uint4*>(out));
   return cudaGetLastError();
 }

@@ -58,6 +58,7 @@ struct GemmParams {
   int rows_total;  // rows of A and C: no tile reads or writes past it
   void* C;
   int ldc;  // output row length in elements
+  int out_f32;  // store epilogues: 1 = fp32 C, 0 = bf16 C
   float* C_scales;
   int ld_cscales;
   float* debug_h;
@@ -342,21 +343,31 @@ __global__ void __launch_bounds__(192, 1)
         tc_fence_after();
         const uint32_t tb = lane_base + static_cast<uint32_t>(acc * BN);
         if constexpr (kMode == kModeStore) {
-          __nv_bfloat16* C = static_cast<__nv_bfloat16*>(p.C);
 #pragma unroll 1
           for (int c = 0; c < BN / 32; ++c) {
             uint32_t v[32];
             tmem_ld32(tb + c * 32, v);
             tmem_ld_wait();
-            uint32_t pk[16];
+            if (p.out_f32) {
+              if (valid) {
+                uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(p.C) + row * p.ldc +
+                                                      ti.nb * BN + c * 32);
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-            if (valid) {
-              uint4* dst = reinterpret_cast<uint4*>(C + row * p.ldc + ti.nb * BN + c * 32);
+                for (int i = 0; i < 8; ++i)
+                  dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+              }
+            } else {
+              uint32_t pk[16];
 #pragma unroll
-              for (int i = 0; i < 4; ++i)
-                dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+              for (int i = 0; i < 16; ++i)
+                pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+              if (valid) {
+                uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.C) +
+                                                      row * p.ldc + ti.nb * BN + c * 32);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                  dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+              }
             }
           }
         } else if constexpr (kMode == kModeSwiglu) {
@@ -477,14 +488,22 @@ __global__ void __launch_bounds__(192, 1)
         }
         if (!ok) break;
         if (valid) {
-          __nv_bfloat16* C = static_cast<__nv_bfloat16*>(p.C);
-          uint4* dst = reinterpret_cast<uint4*>(C + row * p.ldc + ti.nb * BN);
+          if (p.out_f32) {
+            float4* dst =
+                reinterpret_cast<float4*>(static_cast<float*>(p.C) + row * p.ldc + ti.nb * BN);
 #pragma unroll
-          for (int i = 0; i < BN / 8; ++i)
-            dst[i] = make_uint4(pack_bf16x2(accv[8 * i], accv[8 * i + 1]),
-                                pack_bf16x2(accv[8 * i + 2], accv[8 * i + 3]),
-                                pack_bf16x2(accv[8 * i + 4], accv[8 * i + 5]),
-                                pack_bf16x2(accv[8 * i + 6], accv[8 * i + 7]));
+            for (int i = 0; i < BN / 4; ++i)
+              dst[i] = make_float4(accv[4 * i], accv[4 * i + 1], accv[4 * i + 2], accv[4 * i + 3]);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.C) + row * p.ldc +
+                                                  ti.nb * BN);
+#pragma unroll
+            for (int i = 0; i < BN / 8; ++i)
+              dst[i] = make_uint4(pack_bf16x2(accv[8 * i], accv[8 * i + 1]),
+                                  pack_bf16x2(accv[8 * i + 2], accv[8 * i + 3]),
+                                  pack_bf16x2(accv[8 * i + 4], accv[8 * i + 5]),
+                                  pack_bf16x2(accv[8 * i + 6], accv[8 * i + 7]));
+          }
         }
       }
     }
@@ -582,6 +601,7 @@ static cudaError_t run_gemm(const GemmLaunch& L, cudaStream_t stream) {
   p.C = L.C;
   const int out_n = Cfg::kSwiglu ? L.N / 2 : L.N;
   p.ldc = out_n;
+  p.out_f32 = L.out_f32;
   p.C_scales = L.C_scales;
   p.ld_cscales = out_n / 128;
   p.debug_h = L.debug_h;

@@ -27,6 +27,7 @@ struct GemmLaunch {
   const int32_t* idx_for_bx = nullptr;
   int M_blk = 0;  // length of idx_for_bx (grouped mode)
   void* C = nullptr;
+  int out_f32 = 0;  // store modes: fp32 C instead of bf16
   float* C_scales = nullptr;
   float* debug_h = nullptr;
   int32_t* status = nullptr;
@@ -46,8 +47,9 @@ cudaError_t launch_tables(const int32_t* ids, int P, int E, int padding_M, int M
 cudaError_t launch_gather_rows(const void* hidden, const int32_t* pair_of_row, int P, int k,
                                int H, void* x_perm, cudaStream_t stream);
 
-cudaError_t launch_unpermute(const void* y, const int32_t* row_of_pair, const float* weights,
-                             int T, int k, int H, float scale, const void* addend, void* out,
+// y fp32 [T*k, H]; addend fp32 [T, H] or null; out bf16 [T, H]
+cudaError_t launch_unpermute(const float* y, const int32_t* row_of_pair, const float* weights,
+                             int T, int k, int H, float scale, const float* addend, void* out,
                              cudaStream_t stream);
 
 cudaError_t launch_swiglu_quant(int M, int F, const void* gate_up, const float* h, int out_fp8,

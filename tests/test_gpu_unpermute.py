@@ -1,0 +1,42 @@
+"""GPU parity of a7, the weighted unpermute (moe_unpermute), against the
+oracle: fp32 y rows gathered by row_of_pair, weighted in slot order, scaled by
+routed_scaling_factor, plus the optional addend, one bf16 cast."""
+import numpy as np
+import pytest
+import torch
+
+from moe_inputs import get_config
+from oracle import moe_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from tests.gpu_util import ensure_built
+    ensure_built()
+
+
+@pytest.mark.parametrize("T,E,k,H,scale,addend", [(9, 4, 2, 128, 1.0, False),
+                                                   (300, 16, 8, 2048, 2.5, True),
+                                                   (77, 7, 3, 7168, 2.827, False)])
+def test_unpermute(T, E, k, H, scale, addend):
+    from tests import gpu_util as gu
+    import moe_routed_expert_top_b200 as M
+    cfg = get_config("tiny", T=T, E=E, top_k=k, H=H, F=64)
+    rng = np.random.default_rng(T)
+    ids = gu.random_ids(T, E, k, rng)
+    _, w = O.route_topk(rng.standard_normal((T, E)).astype(np.float32), k, O.SIGMOID, True)
+    L, tables, status, _ = gu.gpu_tables(cfg, ids)
+    ref_t = O.dispatch_tables(ids, E, 128)
+    y = (rng.standard_normal((T * k, H)) * 1.5).astype(np.float32)
+    add = (rng.standard_normal((T, H))).astype(np.float32) if addend else None
+    out = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+    M.moe_unpermute(gu.problem(cfg), torch.from_numpy(y).cuda(), tables, torch.from_numpy(w).cuda(),
+                    scale, torch.from_numpy(add).cuda() if addend else None, out)
+    torch.cuda.synchronize()
+    ref = O.unpermute(y, ref_t["row_of_pair"], w, scale, addend=add)
+    gu.assert_within_tol(gu.f64(out), ref, "unpermute")
+    # one bf16 cast of an fp32 sum: within one bf16 ulp of the exact value
+    exact = O.unpermute(y, ref_t["row_of_pair"], w, scale, addend=add, round_output=False)
+    assert np.all(np.abs(gu.f64(out) - exact) <= np.abs(exact) * 2.0 ** -7 + 1e-6)
