@@ -244,6 +244,39 @@ moe_status moe_experts_forward(const moe_problem* prob, const void* hidden,
                                float scale, void* out, void* workspace, size_t ws_bytes,
                                moe_stream_t stream);
 
+/* Capacity of the library's built-in scratch area used by
+ * moe_experts_forward_noalloc: 64 MiB of device memory. */
+#define MOE_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+/* moe_experts_forward without a caller-supplied workspace: the pages have no
+ * counterpart; this exists for callers that cannot allocate device memory.
+ * Some callers have no way to obtain a scratch buffer: a plug-in running
+ * inside a host program that owns every device allocation through its own
+ * allocator and forbids others, or a service whose device-memory budget is
+ * fixed when it starts. This call takes the same arguments as
+ * moe_experts_forward minus (workspace, ws_bytes) and keeps its workspace in a
+ * file-scope device array of MOE_NOALLOC_SCRATCH_BYTES bytes inside the
+ * library; every GPU that loads the library holds that array until the
+ * process exits.
+ *   - It allocates nothing: no cudaMalloc, cudaFree or allocating library
+ *     routine. Its first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make
+ *     that first call before any stream capture.
+ *   - Problems whose moe_workspace_bytes() exceeds MOE_NOALLOC_SCRATCH_BYTES
+ *     are rejected with MOE_ERR_WORKSPACE before anything is enqueued.
+ *   - All calls share the one array and it keeps the last call's contents;
+ *     the call itself clears what must start at zero (the status word).
+ *     Calls whose work overlaps on the GPU (different streams, or different
+ *     host threads on one device) race on the array: serialise them.
+ *   - The device status word is the array's first int32; it is not readable
+ *     through this interface, so device-side flags are not reported here. */
+moe_status moe_experts_forward_noalloc(const moe_problem* prob, const void* hidden,
+                                       const int32_t* topk_ids, const float* topk_weights,
+                                       const void* w_gate_up, const void* w_down,
+                                       const float* w_down_scales,
+                                       const void* ws_gate_up, const void* ws_down,
+                                       float scale, void* out, moe_stream_t stream);
+
 /* Maps a device status word (copied to the host after a sync) to a status:
  * MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_DEVICE_FLAG. */
 moe_status moe_decode_device_status(int32_t dev_status);

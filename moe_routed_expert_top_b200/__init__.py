@@ -37,7 +37,7 @@ EXPORTED_SYMBOLS = (
     "moe_get_tables_layout", "moe_workspace_bytes", "moe_route_topk", "moe_route_permute",
     "moe_grouped_gemm", "moe_swiglu_quant", "moe_unpermute", "moe_quantize_weight_128x128",
     "moe_experts_forward", "moe_decode_device_status", "moe_status_string",
-    "moe_last_cuda_error", "moe_last_launch_count",
+    "moe_last_cuda_error", "moe_last_launch_count", "moe_experts_forward_noalloc",
 )
 
 
@@ -109,6 +109,8 @@ def lib() -> ctypes.CDLL:
                                                        ctypes.c_int32, _P, _P, _P, _P]),
         "moe_experts_forward": (ctypes.c_int, [PP, _P, _P, _P, _P, _P, _P, _P, _P,
                                                ctypes.c_float, _P, _P, ctypes.c_size_t, _P]),
+        "moe_experts_forward_noalloc": (ctypes.c_int, [PP, _P, _P, _P, _P, _P, _P, _P, _P,
+                                                       ctypes.c_float, _P, _P]),
         "moe_decode_device_status": (ctypes.c_int, [ctypes.c_int32]),
         "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "moe_last_cuda_error": (ctypes.c_char_p, []),
