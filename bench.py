@@ -248,16 +248,31 @@ def run_b200(args, cfg, rank, world, device):
     torch.cuda.synchronize()
     assert layer.device_status() == 0, "device status flag set"
     launches_per_step = M.moe_last_launch_count()
+    # eager: one C call per step (its launches go out one by one)
+    eager = time_steps(step, max(3, min(args.steps, 50)), flush, stream)
+    eager_ms = max_over_ranks(sum(eager) / len(eager), world, device)
+    timed = step
+    if not args.no_graph:
+        # the same forward captured once as a CUDA graph and replayed per step
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        torch.cuda.synchronize()
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+        timed = graph.replay
 
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
                       else int(os.environ.get("LOCAL_RANK", 0))) as clk:
         t0 = time.perf_counter()
-        times = time_steps(step, args.steps, flush, stream)
+        times = time_steps(timed, args.steps, flush, stream)
         torch.cuda.synchronize()
         wall = time.perf_counter() - t0
     barrier(world)
+    assert layer.device_status() == 0, "device status flag set"
     ms = sum(times) / len(times)
     ms = max_over_ranks(ms, world, device)
     clocks = clk.summary()
@@ -331,6 +346,9 @@ def run_b200(args, cfg, rank, world, device):
                    "parallelism": f"replicas x{world}"},
         "roofline": roof, "forward_roofline": fwd_roof,
         "stages_ms": {k: round(v, 4) for k, v in stages.items()},
+        "launch": "cuda graph replay of moe_experts_forward" if not args.no_graph
+                  else "eager moe_experts_forward calls",
+        "eager_ms": round(eager_ms, 4),
         "e2e": {"value": round(e2e_ms, 4), "unit": "ms/layer", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
@@ -481,9 +499,18 @@ def main(argv=None):
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=20.0)
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time eager calls instead of a CUDA graph replay of the forward")
+    ap.add_argument("--override", default="",
+                    help="workload fields to replace, e.g. E=16,T=256 (small profiling cases)")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
     cfg = get_config(args.config)
+    if args.override:
+        kv = dict(item.split("=", 1) for item in args.override.split(","))
+        typed = {k: (v.lower() in ("1", "true")) if isinstance(getattr(cfg, k), bool)
+                 else type(getattr(cfg, k))(v) for k, v in kv.items()}
+        cfg = cfg.replace(name=cfg.name + "[" + args.override + "]", **typed)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -5,8 +5,8 @@
  *   a1 top-k routing of router logits (softmax or sigmoid scores, optionally
  *      renormalised over the k picks);
  *   a2 the expert-sorted permutation and its dispatch tables (group_sizes,
- *      group_offsets, group_padded_offsets, group_idx_for_bx) from one
- *      histogram + stable scan kernel, with no host synchronisation;
+ *      group_offsets, group_padded_offsets, group_idx_for_bx) from a chunked
+ *      histogram + stable scan on the device, with no host synchronisation;
  *   a3 the permute gather of token rows into expert order;
  *   a4 a persistent grouped gate+up GEMM on tcgen05 tensor cores (TMEM
  *      accumulators, TMA loads whose out-of-bounds zero fill covers ragged
@@ -121,7 +121,9 @@ typedef struct moe_problem {
  *   row_of_pair[P]            permuted row of flat pair p = t*k + j; experts in
  *                             index order, pairs of one expert in flat order
  *   pair_of_row[P]            inverse permutation (-1 for rows left empty by
- *                             out-of-range ids) */
+ *                             out-of-range ids)
+ *   chunk_counts[...]         scratch of the table builder (per-chunk expert
+ *                             counts); contents unspecified */
 typedef struct moe_tables_layout {
   int64_t group_sizes;
   int64_t group_offsets;
@@ -129,6 +131,7 @@ typedef struct moe_tables_layout {
   int64_t group_idx_for_bx;
   int64_t row_of_pair;
   int64_t pair_of_row;
+  int64_t chunk_counts;
   int64_t total_int32;  /* elements the buffer must hold */
   int32_t M_blk;
   int32_t P;

@@ -68,7 +68,7 @@ class TablesLayout(ctypes.Structure):
         ("group_sizes", ctypes.c_int64), ("group_offsets", ctypes.c_int64),
         ("group_padded_offsets", ctypes.c_int64), ("group_idx_for_bx", ctypes.c_int64),
         ("row_of_pair", ctypes.c_int64), ("pair_of_row", ctypes.c_int64),
-        ("total_int32", ctypes.c_int64), ("M_blk", ctypes.c_int32), ("P", ctypes.c_int32),
+        ("chunk_counts", ctypes.c_int64), ("total_int32", ctypes.c_int64), ("M_blk", ctypes.c_int32), ("P", ctypes.c_int32),
     ]
 
 

@@ -69,6 +69,8 @@ void fill_layout(const moe_problem* pr, moe_tables_layout* L) {
   o += round_up(P, 4);
   L->pair_of_row = o;
   o += round_up(P, 4);
+  L->chunk_counts = o;
+  o += round_up(static_cast<int64_t>(moe::tables_num_chunks(static_cast<int>(P))) * E, 4);
   L->total_int32 = o;
   L->M_blk = static_cast<int32_t>(M_blk);
   L->P = static_cast<int32_t>(P);
@@ -152,7 +154,8 @@ moe_status moe_route_permute(const moe_problem* prob, const float* logits, int32
   MOE_CUDA_TRY(moe::launch_tables(topk_ids, L.P, prob->E, prob->padding_M, L.M_blk,
                                   tables + L.group_sizes, tables + L.group_offsets,
                                   tables + L.group_padded_offsets, tables + L.group_idx_for_bx,
-                                  tables + L.row_of_pair, tables + L.pair_of_row, dev_status, st));
+                                  tables + L.row_of_pair, tables + L.pair_of_row,
+                                  tables + L.chunk_counts, dev_status, st));
   if (hidden != nullptr)
     MOE_CUDA_TRY(moe::launch_gather_rows(hidden, tables + L.pair_of_row, L.P, prob->top_k,
                                          prob->H, x_perm, st));
@@ -317,7 +320,8 @@ moe_status moe_experts_forward(const moe_problem* prob, const void* hidden,
   MOE_CUDA_TRY(moe::launch_tables(topk_ids, L.P, E, prob->padding_M, L.M_blk,
                                   tables + L.group_sizes, tables + L.group_offsets,
                                   tables + L.group_padded_offsets, tables + L.group_idx_for_bx,
-                                  tables + L.row_of_pair, tables + L.pair_of_row, status, st));
+                                  tables + L.row_of_pair, tables + L.pair_of_row,
+                                  tables + L.chunk_counts, status, st));
   MOE_CUDA_TRY(moe::launch_gather_rows(hidden, tables + L.pair_of_row, L.P, k, H, x_perm, st));
   g_last_launches += 2;
 

@@ -31,20 +31,44 @@ __global__ void __launch_bounds__(128) unpermute_kernel(const float4* __restrict
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
   const int64_t pbase = static_cast<int64_t>(t) * k;
-  for (int j = 0; j < k; ++j) {
-    const int row = __ldg(row_of_pair + pbase + j);
-    if (row < 0 || row >= P) continue;
-    const float wt = __ldg(w + pbase + j);
-    const float4* src = y + (static_cast<int64_t>(row) * H8 + c) * 2;
-    const float4 a = __ldg(src), b = __ldg(src + 1);
-    acc[0] = fmaf(wt, a.x, acc[0]);
-    acc[1] = fmaf(wt, a.y, acc[1]);
-    acc[2] = fmaf(wt, a.z, acc[2]);
-    acc[3] = fmaf(wt, a.w, acc[3]);
-    acc[4] = fmaf(wt, b.x, acc[4]);
-    acc[5] = fmaf(wt, b.y, acc[5]);
-    acc[6] = fmaf(wt, b.z, acc[6]);
-    acc[7] = fmaf(wt, b.w, acc[7]);
+  // slots in groups of 8: all row indices, then all loads, then the FMAs in
+  // slot order, so each thread keeps 16 independent 16-byte loads in flight
+  for (int j0 = 0; j0 < k; j0 += 8) {
+    int rows[8];
+    float wts[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const bool in = j0 + j < k;
+      const int r = in ? __ldg(row_of_pair + pbase + j0 + j) : -1;
+      rows[j] = (r >= 0 && r < P) ? r : -1;
+      wts[j] = in ? __ldg(w + pbase + j0 + j) : 0.0f;
+    }
+    float4 va[8], vb[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (rows[j] >= 0) {
+        const float4* src = y + (static_cast<int64_t>(rows[j]) * H8 + c) * 2;
+        va[j] = __ldg(src);
+        vb[j] = __ldg(src + 1);
+      } else {
+        va[j] = vb[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        wts[j] = 0.0f;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (j0 + j >= k) break;
+      if (rows[j] < 0) continue;
+      const float wt = wts[j];
+      acc[0] = fmaf(wt, va[j].x, acc[0]);
+      acc[1] = fmaf(wt, va[j].y, acc[1]);
+      acc[2] = fmaf(wt, va[j].z, acc[2]);
+      acc[3] = fmaf(wt, va[j].w, acc[3]);
+      acc[4] = fmaf(wt, vb[j].x, acc[4]);
+      acc[5] = fmaf(wt, vb[j].y, acc[5]);
+      acc[6] = fmaf(wt, vb[j].z, acc[6]);
+      acc[7] = fmaf(wt, vb[j].w, acc[7]);
+    }
   }
   float v[8];
   if (addend != nullptr) {

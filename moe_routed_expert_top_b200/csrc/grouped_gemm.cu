@@ -624,9 +624,14 @@ cudaError_t launch_grouped_gemm(const GemmLaunch& L, cudaStream_t stream) {
       if (L.N % 256 == 0) return run_gemm<kModeStore, 256>(L, stream);
       if (L.N % 128 == 0) return run_gemm<kModeStore, 128>(L, stream);
       return run_gemm<kModeStore, 64>(L, stream);
-    case kModeSwiglu:
-      if ((L.N / 2) % 128 == 0) return run_gemm<kModeSwiglu, 256>(L, stream);
+    case kModeSwiglu: {
+      // Small expert groups (decode): every tile streams its full weight slab,
+      // so 64-column h tiles halve the tile cost and cut the idle tail of the
+      // last wave of the persistent grid.
+      const bool small_groups = L.group_padded != nullptr && L.rows < 64 * L.E;
+      if ((L.N / 2) % 128 == 0 && !small_groups) return run_gemm<kModeSwiglu, 256>(L, stream);
       return run_gemm<kModeSwiglu, 128>(L, stream);
+    }
     case kModeSwigluFp8:
       return run_gemm<kModeSwigluFp8, 256>(L, stream);
     case kModeFp8Store:

@@ -39,10 +39,12 @@ cudaError_t launch_grouped_gemm(const GemmLaunch& L, cudaStream_t stream);
 cudaError_t launch_route_topk(const float* logits, int T, int E, int k, int score_fn,
                               int renormalize, int32_t* ids, float* weights, cudaStream_t stream);
 
+// chunk_counts: scratch of tables_num_chunks(P) * E int32
 cudaError_t launch_tables(const int32_t* ids, int P, int E, int padding_M, int M_blk,
                           int32_t* sizes, int32_t* offsets, int32_t* padded, int32_t* idx_for_bx,
-                          int32_t* row_of_pair, int32_t* pair_of_row, int32_t* status,
-                          cudaStream_t stream);
+                          int32_t* row_of_pair, int32_t* pair_of_row, int32_t* chunk_counts,
+                          int32_t* status, cudaStream_t stream);
+int tables_num_chunks(int P);
 
 cudaError_t launch_gather_rows(const void* hidden, const int32_t* pair_of_row, int P, int k,
                                int H, void* x_perm, cudaStream_t stream);

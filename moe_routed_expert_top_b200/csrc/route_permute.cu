@@ -1,5 +1,5 @@
-// route_permute.cu - a1 top-k routing, a2 dispatch tables + stable
-// permutation, a3 permute gather.
+// route_permute.cu - a1 top-k routing and a3 the permute gather (a2, the
+// dispatch tables, is in tables.cu).
 //
 // Built with --fmad=false: the routing weights use only explicitly rounded
 // float32 operations (__fmul_rn / __fadd_rn / __fsub_rn / __fdiv_rn), so they
@@ -128,168 +128,6 @@ cudaError_t launch_route_topk(const float* logits, int T, int E, int k, int scor
   const int warps = 8;
   route_topk_kernel<<<(T + warps - 1) / warps, warps * 32, 0, stream>>>(
       logits, T, E, k, score_fn, renormalize, ids, weights);
-  return cudaGetLastError();
-}
-
-// ---------------------------------------------------------------------------
-// a2: histogram + stable scan -> tables and permutation (one CTA, no host sync)
-// ---------------------------------------------------------------------------
-// The P pairs are cut into 32 contiguous segments, one per warp. Pass 1: each
-// warp counts its segment per expert (32 pairs at a time; __match_any_sync
-// groups equal ids, the group's lowest lane adds the group size). A per-expert
-// scan over the 32 warp counts and a block scan over experts give every
-// (warp, expert) its first row. Pass 2: each warp walks its segment again in
-// order; a pair's row is its (warp, expert) base plus the number of earlier
-// lanes in its match group. Rows therefore follow flat pair order inside each
-// expert (a stable sort by expert).
-
-__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int o = __shfl_up_sync(0xffffffffu, v, off);
-    if (lane >= off) v += o;
-  }
-  return v;
-}
-
-__global__ void __launch_bounds__(1024) tables_kernel(
-    const int32_t* __restrict__ ids, int P, int E, int pad, int M_blk, int32_t* __restrict__ sizes,
-    int32_t* __restrict__ offsets, int32_t* __restrict__ padded, int32_t* __restrict__ idx_for_bx,
-    int32_t* __restrict__ row_of_pair, int32_t* __restrict__ pair_of_row,
-    int32_t* __restrict__ status) {
-  extern __shared__ int smem[];
-  int* hist = smem;                  // [32][E]: per-warp counts, then bases
-  int* s_off = hist + 32 * E;        // [E + 1]
-  int* s_pad = s_off + E + 1;        // [E + 1]
-  int* s_tot = s_pad + E + 1;        // [2][32] warp totals of the two scans
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5;
-  const int lane = tid & 31;
-  for (int i = tid; i < 32 * E; i += blockDim.x) hist[i] = 0;
-  __syncthreads();
-
-  const int seg = (P + 31) / 32;
-  const int beg = warp * seg;
-  const int end = min(P, beg + seg);
-  bool bad = false;
-  for (int base = beg; base < end; base += 32) {
-    const int p = base + lane;
-    int id = -1;
-    if (p < end) {
-      id = __ldg(ids + p);
-      if (id < 0 || id >= E) {
-        bad = true;
-        id = -1;
-      }
-    }
-    const unsigned mask = __match_any_sync(0xffffffffu, id);
-    if (id >= 0 && lane == __ffs(mask) - 1) hist[warp * E + id] += __popc(mask);
-    __syncwarp();
-  }
-  if (bad) atomicOr(status, MOE_DEV_BAD_EXPERT_ID_FLAG);
-  __syncthreads();
-
-  // per expert: exclusive scan over warps (in place), total size
-  int size = 0;
-  if (tid < E) {
-    for (int w = 0; w < 32; ++w) {
-      const int c = hist[w * E + tid];
-      hist[w * E + tid] = size;
-      size += c;
-    }
-  }
-  const int padsz = (size + pad - 1) / pad * pad;
-  // block exclusive scans of size and padded size over experts (E <= 1024)
-  const int inc_s = warp_incl_scan(size, lane);
-  const int inc_p = warp_incl_scan(padsz, lane);
-  if (lane == 31) {
-    s_tot[warp] = inc_s;
-    s_tot[32 + warp] = inc_p;
-  }
-  __syncthreads();
-  if (warp == 0) {
-    const int a = warp_incl_scan(s_tot[lane], lane);
-    const int b = warp_incl_scan(s_tot[32 + lane], lane);
-    __syncwarp();
-    s_tot[lane] = a;
-    s_tot[32 + lane] = b;
-  }
-  __syncthreads();
-  const int ex_s = inc_s - size + (warp > 0 ? s_tot[warp - 1] : 0);
-  const int ex_p = inc_p - padsz + (warp > 0 ? s_tot[32 + warp - 1] : 0);
-  if (tid < E) {
-    s_off[tid] = ex_s;
-    s_pad[tid] = ex_p;
-    sizes[tid] = size;
-    offsets[tid] = ex_s;
-    padded[tid] = ex_p;
-    if (tid == E - 1) {
-      s_off[E] = ex_s + size;
-      s_pad[E] = ex_p + padsz;
-      offsets[E] = ex_s + size;
-      padded[E] = ex_p + padsz;
-    }
-  }
-  __syncthreads();
-  if (tid < E) {
-    for (int w = 0; w < 32; ++w) hist[w * E + tid] += s_off[tid];
-  }
-  __syncthreads();
-
-  for (int base = beg; base < end; base += 32) {
-    const int p = base + lane;
-    int id = -1;
-    if (p < end) {
-      id = __ldg(ids + p);
-      if (id < 0 || id >= E) id = -1;
-    }
-    const unsigned mask = __match_any_sync(0xffffffffu, id);
-    const int rank = __popc(mask & ((1u << lane) - 1u));
-    if (id >= 0) {
-      const int row = hist[warp * E + id] + rank;
-      row_of_pair[p] = row;
-      pair_of_row[row] = p;
-    } else if (p < end) {
-      row_of_pair[p] = -1;
-    }
-    __syncwarp();
-    if (id >= 0 && lane == __ffs(mask) - 1) hist[warp * E + id] += __popc(mask);
-    __syncwarp();
-  }
-  // rows left empty by skipped (out-of-range) pairs
-  for (int r = s_off[E] + tid; r < P; r += blockDim.x) pair_of_row[r] = -1;
-
-  // M-block -> expert: largest g with padded[g] <= bx * pad
-  for (int bx = tid; bx < M_blk; bx += blockDim.x) {
-    const long long x = static_cast<long long>(bx) * pad;
-    int lo = 0, hi = E - 1;  // s_pad[0] = 0 <= x
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (s_pad[mid] <= x)
-        lo = mid;
-      else
-        hi = mid - 1;
-    }
-    idx_for_bx[bx] = lo;
-  }
-}
-
-cudaError_t launch_tables(const int32_t* ids, int P, int E, int padding_M, int M_blk,
-                          int32_t* sizes, int32_t* offsets, int32_t* padded, int32_t* idx_for_bx,
-                          int32_t* row_of_pair, int32_t* pair_of_row, int32_t* status,
-                          cudaStream_t stream) {
-  const size_t smem = (static_cast<size_t>(32) * E + 2 * (E + 1) + 64) * sizeof(int);
-  static bool attr_done[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (smem > 48 * 1024 && dev >= 0 && dev < 64 && !attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(tables_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(32 * 1024 * 4 + 2 * 1025 * 4 + 64 * 4));
-    if (e != cudaSuccess) return e;
-    attr_done[dev] = true;
-  }
-  tables_kernel<<<1, 1024, smem, stream>>>(ids, P, E, padding_M, M_blk, sizes, offsets, padded,
-                                           idx_for_bx, row_of_pair, pair_of_row, status);
   return cudaGetLastError();
 }
 
