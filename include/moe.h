@@ -95,6 +95,17 @@ enum {
   MOE_EPI_STORE_F32 = 3    /* C fp32 [rows, N] = A @ B^T (the accumulator, unrounded) */
 };
 
+/* Tiling choice, OR-ed into moe_grouped_gemm's `epilogue` argument. Both
+ * compute the same result.
+ *   MOE_TILE_AUTO        the library's choice (weight rows where supported)
+ *   MOE_TILE_TOKEN_ROWS  128 token rows x N columns per tile (every epilogue)
+ *   MOE_TILE_WEIGHT_ROWS 128 weight rows x (the expert's tokens, <= 256, rounded
+ *                        up to 16) per tile: MMA work follows the real group
+ *                        sizes; bf16 mode with MOE_EPI_STORE / STORE_F32
+ *                        (N % 128 == 0) or MOE_EPI_SWIGLU (N % 128 == 0) only,
+ *                        else MOE_ERR_UNSUPPORTED. */
+enum { MOE_TILE_AUTO = 0x00, MOE_TILE_TOKEN_ROWS = 0x10, MOE_TILE_WEIGHT_ROWS = 0x20 };
+
 /* One MoE layer's shape and routing options. */
 typedef struct moe_problem {
   int32_t T;            /* tokens (>= 0; 0 is a no-op) */

@@ -174,6 +174,10 @@ moe_status moe_grouped_gemm(const moe_problem* prob, int32_t M_rows, int32_t N, 
   const bool fp8 = A_scales != nullptr || B_scales != nullptr;
   if (fp8 && (A_scales == nullptr || B_scales == nullptr)) return MOE_ERR_INVALID_ARG;
   moe::GemmLaunch g;
+  const int tiling = (epilogue >> 4) & 0xF;
+  epilogue &= 0xF;
+  if (tiling > moe::kTilingWeights) return MOE_ERR_INVALID_ARG;
+  g.tiling = tiling;
   if (tables != nullptr) {
     moe_status s = check_problem(prob, false);
     if (s != MOE_OK) return s;
@@ -231,6 +235,8 @@ moe_status moe_grouped_gemm(const moe_problem* prob, int32_t M_rows, int32_t N, 
   g.C_scales = C_scales;
   g.debug_h = debug_h;
   g.status = dev_status;
+  if (g.tiling == moe::kTilingWeights && !moe::grouped_gemm_t_supported(g))
+    return MOE_ERR_UNSUPPORTED;
   MOE_CUDA_TRY(moe::launch_grouped_gemm(g, reinterpret_cast<cudaStream_t>(stream)));
   return MOE_OK;
 }

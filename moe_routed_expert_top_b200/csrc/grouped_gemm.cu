@@ -619,6 +619,10 @@ static cudaError_t run_gemm(const GemmLaunch& L, cudaStream_t stream) {
 }
 
 cudaError_t launch_grouped_gemm(const GemmLaunch& L, cudaStream_t stream) {
+  if (grouped_gemm_t_supported(L) &&
+      (L.tiling == kTilingWeights || (L.tiling == kTilingAuto && grouped_gemm_t_preferred(L))))
+    return launch_grouped_gemm_t(L, stream);
+  if (L.tiling == kTilingWeights) return cudaErrorNotSupported;
   switch (L.mode) {
     case kModeStore:
       if (L.N % 256 == 0) return run_gemm<kModeStore, 256>(L, stream);

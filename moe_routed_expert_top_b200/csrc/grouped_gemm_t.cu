@@ -1,0 +1,515 @@
+// grouped_gemm_t.cu - the grouped GEMM with weights on the MMA's M side
+// ("transposed" tiles): D^T[w, t] = sum_k W[e][w, k] * X[t, k].
+//
+// Same operation as grouped_gemm.cu (TileOPs PR #1580 "Grouped-GEMM TMA OOB
+// zero-fill + unpermute out=", Grouped-GEMM kernel: C[e] = A[e] @ B[e]^T over
+// each expert's rows), tiled the other way round: a tile is 128 weight rows x
+// up to TN token rows of one expert. The MMA's N is the tile's token count
+// rounded up to 16, so the tensor work follows the real group sizes instead of
+// padding every expert to 128-row blocks, and a small group (decode) loads
+// only as many token rows as it has (TMA boxes of 32/64/128/256 rows).
+//
+// Tiles are ordered (expert, weight block, token chunk), token chunks
+// innermost, so the chunks that share a weight block run at the same time and
+// read it once from HBM. Empty experts own no tile (pypto-lib PR #809).
+//
+// Modes:
+//   store  : C [rows, N] (fp32 or bf16) = X @ W[e]^T; weight block = 128 rows.
+//   swiglu : h bf16 [rows, F] = SiLU(G[:, :F]) * G[:, F:], G = X @ W[e]^T with
+//            W[e] = [gate rows; up rows] (TileOPs PR #778, Design); a weight
+//            block stacks 64 gate rows over the matching 64 up rows, so one
+//            M=128 MMA produces both and the epilogue pairs lane r with lane
+//            r + 64 through shared memory (XTuner PR #2089, SiLU(gate)*up).
+// Warp roles and the bounded-wait/teardown protocol are those of
+// grouped_gemm.cu: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer,
+// warps 2-5 epilogue (TMEM lane = weight row), two TMEM accumulators.
+// The epilogue stages 32 token rows at a time in shared memory and writes
+// them row-major with 16-byte stores, masking rows past the tile's tokens.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace moe {
+
+namespace {
+
+enum TMode { kTStore = 0, kTSwiglu = 1 };
+
+constexpr int kXBoxes = 4;  // token-tile TMA boxes of 32, 64, 128, 256 rows
+
+struct TParams {
+  int M_dense;  // rows in dense mode (group tables null)
+  int N;        // rows of W per expert
+  int K;
+  int E;
+  const int32_t* group_sizes;
+  const int32_t* group_offsets;
+  int rows_total;
+  void* C;
+  int ldc;      // output row length in elements
+  int out_f32;  // store mode: fp32 C
+  int32_t* status;
+};
+
+__host__ __device__ constexpr int tmin(int a, int b) { return a < b ? a : b; }
+
+template <int kMode, int TN>
+struct TCfg {
+  static constexpr int BK = 64;           // bf16 elements per 128-byte smem row
+  static constexpr int K_STEPS = 4;       // MMAs (K=16) per stage
+  static constexpr int A_BYTES = 128 * 128;     // weight tile: 128 rows x 128 B
+  static constexpr int B_BYTES = TN * 128;      // token tile: up to TN rows x 128 B
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = tmin(8, (200 * 1024) / STAGE_BYTES);
+  static constexpr int NUM_ACC = 2;
+  static constexpr int TMEM_COLS = 2 * TN;      // TN <= 256
+  static constexpr int STAGE_OUT_BYTES = 32 * 128 * 4;  // 32 token rows x 128 fp32
+  static constexpr int NUM_BARS = 2 * STAGES + 2 * NUM_ACC + 1;
+  static constexpr int MAX_E = 1024;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STAGE_OUT_BYTES +
+                                    NUM_BARS * 8 + 16 + (MAX_E + 8) * 4;
+  static constexpr int WROWS = (kMode == kTSwiglu) ? 64 : 128;  // output columns per tile
+  static_assert(TN % 32 == 0 && TN >= 32 && TN <= 256, "token tile");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+};
+
+struct TTile {
+  int e, wb, m0, nt;
+};
+
+// Tile t -> (expert, weight block, token chunk). cpre[e] = token chunks of the
+// experts before e (shared memory, built at kernel start); WB weight blocks.
+__device__ __forceinline__ bool t_decode(const TParams& p, const int* cpre, int E, int WB, int TN,
+                                         int t, TTile& ti) {
+  int lo = 0, hi = E - 1;  // largest e with WB*cpre[e] <= t
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (WB * cpre[mid] <= t)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  const int e = lo;
+  const int chunks = cpre[e + 1] - cpre[e];
+  if (chunks <= 0) return false;
+  const int local = t - WB * cpre[e];
+  const int wb = local / chunks;
+  const int c = local - wb * chunks;
+  const int size = p.group_sizes ? __ldg(p.group_sizes + e) : p.M_dense;
+  const int off = p.group_offsets ? __ldg(p.group_offsets + e) : 0;
+  ti.e = e;
+  ti.wb = wb;
+  ti.m0 = off + c * TN;
+  ti.nt = tmin(TN, size - c * TN);
+  if (ti.nt <= 0 || ti.m0 < 0 || ti.m0 + ti.nt > p.rows_total) {
+    if (threadIdx.x == 0 && ti.nt > 0) atomicOr(p.status, MOE_DEV_BAD_TABLES_FLAG);
+    return false;
+  }
+  return true;
+}
+
+__device__ __forceinline__ int xbox_for(int n) {  // smallest box (32/64/128/256) holding n rows
+  return n <= 32 ? 0 : n <= 64 ? 1 : n <= 128 ? 2 : 3;
+}
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
+
+template <int kMode, int TN>
+__global__ void __launch_bounds__(192, 1)
+    grouped_gemm_t_kernel(const __grid_constant__ CUtensorMap tmW,
+                          const __grid_constant__ CUtensorMap tmX0,
+                          const __grid_constant__ CUtensorMap tmX1,
+                          const __grid_constant__ CUtensorMap tmX2,
+                          const __grid_constant__ CUtensorMap tmX3, const TParams p) {
+  using Cfg = TCfg<kMode, TN>;
+  constexpr int STAGES = Cfg::STAGES;
+  constexpr int NUM_ACC = Cfg::NUM_ACC;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;                                   // weight tiles
+  uint8_t* sB = smem + STAGES * Cfg::A_BYTES;           // token tiles
+  float* sOut = reinterpret_cast<float*>(sB + STAGES * Cfg::B_BYTES);  // [32][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sOut) +
+                                               Cfg::STAGE_OUT_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NUM_BARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // set only by epilogue threads, read only after their shared barrier: the four
+  // epilogue warps always agree on whether to stop
+  volatile int* epi_abort = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  int* cpre = reinterpret_cast<int*>(tmem_slot + 4);  // [E + 1]
+
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = full0 + 8 * STAGES;
+  const uint32_t tfull0 = empty0 + 8 * STAGES;
+  const uint32_t tempty0 = tfull0 + 8 * NUM_ACC;
+  const uint32_t drain_bar = tempty0 + 8 * NUM_ACC;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int E = p.group_sizes ? p.E : 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int a = 0; a < NUM_ACC; ++a) {
+      mbar_init(tfull0 + 8 * a, 1);
+      mbar_init(tempty0 + 8 * a, 4);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    *epi_abort = 0;
+    mbar_fence_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmX0);
+    tma_prefetch_desc(&tmX1);
+    tma_prefetch_desc(&tmX2);
+    tma_prefetch_desc(&tmX3);
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), Cfg::TMEM_COLS);
+  // token chunks per expert -> exclusive prefix cpre[0..E] (192 threads)
+  {
+    const int per = (E + 191) / 192;
+    const int beg = threadIdx.x * per;
+    int local = 0;
+    for (int i = 0; i < per && beg + i < E; ++i) {
+      const int s = p.group_sizes ? __ldg(p.group_sizes + beg + i) : p.M_dense;
+      local += (s + TN - 1) / TN;
+    }
+    int inc = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, inc, off);
+      if (lane >= off) inc += o;
+    }
+    int* wsum = reinterpret_cast<int*>(sOut);  // scratch before the epilogue uses it
+    if (lane == 31) wsum[warp] = inc;
+    __syncthreads();
+    int before = 0;
+    for (int w = 0; w < warp; ++w) before += wsum[w];
+    int run = before + inc - local;
+    for (int i = 0; i < per && beg + i < E; ++i) {
+      cpre[beg + i] = run;
+      const int s = p.group_sizes ? __ldg(p.group_sizes + beg + i) : p.M_dense;
+      run += (s + TN - 1) / TN;
+    }
+    if (threadIdx.x == 191) cpre[E] = before + inc;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int WB = (kMode == kTSwiglu) ? (p.N / 2) / 64 : p.N / 128;
+  const int total_tiles = WB * cpre[E];
+  const int KB = p.K / Cfg::BK;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol_act = l2_policy_evict_last();
+      const uint64_t pol_w = l2_policy_evict_first();
+      const CUtensorMap* xmaps[kXBoxes] = {&tmX0, &tmX1, &tmX2, &tmX3};
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < total_tiles; t += gridDim.x) {
+        TTile ti;
+        if (!t_decode(p, cpre, E, WB, TN, t, ti)) continue;
+        const int nmma = (ti.nt + 15) & ~15;
+        const int xb = xbox_for(nmma);
+        const uint32_t bytes = Cfg::A_BYTES + (32u << xb) * 128u;
+        const int wrow = ti.e * p.N + ti.wb * Cfg::WROWS;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = full0 + 8 * stage;
+          mbar_arrive_expect_tx(fb, bytes);
+          const uint32_t a_dst = smem_u32(sA + stage * Cfg::A_BYTES);
+          if constexpr (kMode == kTSwiglu) {
+            tma_load_2d(a_dst, &tmW, kb * Cfg::BK, wrow, fb, pol_w);                  // gate
+            tma_load_2d(a_dst + 64 * 128, &tmW, kb * Cfg::BK, wrow + p.N / 2, fb, pol_w);  // up
+          } else {
+            tma_load_2d(a_dst, &tmW, kb * Cfg::BK, wrow, fb, pol_w);
+          }
+          tma_load_2d(smem_u32(sB + stage * Cfg::B_BYTES), xmaps[xb], kb * Cfg::BK, ti.m0, fb,
+                      pol_act);
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        const uint32_t n = issued < static_cast<uint32_t>(STAGES) ? issued : STAGES;
+        int s = stage;
+        uint32_t ph = phase;
+        for (uint32_t i = 0; i < n; ++i) {
+          if (--s < 0) {
+            s = STAGES - 1;
+            ph ^= 1u;
+          }
+          mbar_wait_drain(full0 + 8 * s, ph);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < total_tiles; t += gridDim.x) {
+        TTile ti;
+        if (!t_decode(p, cpre, E, WB, TN, t, ti)) continue;
+        const int nmma = (ti.nt + 15) & ~15;
+        const uint32_t idesc = idesc_bf16_f32(128, nmma);
+        if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + static_cast<uint32_t>(acc * TN);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t adesc = smem_desc_sw128(smem_u32(sA + stage * Cfg::A_BYTES));
+          const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + stage * Cfg::B_BYTES));
+#pragma unroll
+          for (int k = 0; k < Cfg::K_STEPS; ++k)
+            mma_bf16(d, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          mma_commit(empty0 + 8 * stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit(tfull0 + 8 * acc);
+        if (++acc == NUM_ACC) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      mma_commit(drain_bar);
+      mbar_wait_drain(drain_bar, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const int r = q * 32 + lane;  // weight row of this thread's TMEM lane
+    const int et = threadIdx.x - 64;  // 0..127 within the epilogue warps
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+      TTile ti;
+      if (!t_decode(p, cpre, E, WB, TN, t, ti)) continue;
+      if (!mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, p.status)) *epi_abort = 1;
+      epi_bar();  // every epilogue warp arrives here whether its wait succeeded or not
+      if (*epi_abort) break;
+      tc_fence_after();
+      const uint32_t tb = lane_base + static_cast<uint32_t>(acc * TN);
+      for (int j0 = 0; j0 < ti.nt; j0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(tb + j0, v);
+        tmem_ld_wait();
+        // sOut[i][r] = D[r][j0 + i]: token row i, weight row r
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sOut[i * 128 + r] = __uint_as_float(v[i]);
+        epi_bar();
+        const int rows = tmin(32, ti.nt - j0);
+        if constexpr (kMode == kTStore) {
+          if (p.out_f32) {
+            // a token row = 128 fp32 = 32 x 16 B; 4 rows per pass
+#pragma unroll
+            for (int pass = 0; pass < 8; ++pass) {
+              const int i = pass * 4 + (et >> 5);
+              const int c4 = et & 31;
+              if (i < rows) {
+                const float4 val = reinterpret_cast<const float4*>(sOut + i * 128)[c4];
+                float* dst = static_cast<float*>(p.C) +
+                             static_cast<int64_t>(ti.m0 + j0 + i) * p.ldc + ti.wb * 128;
+                reinterpret_cast<float4*>(dst)[c4] = val;
+              }
+            }
+          } else {
+            // a token row = 128 bf16 = 16 x 16 B; 8 rows per pass
+#pragma unroll
+            for (int pass = 0; pass < 4; ++pass) {
+              const int i = pass * 8 + (et >> 4);
+              const int c8 = et & 15;
+              if (i < rows) {
+                const float* src = sOut + i * 128 + c8 * 8;
+                const uint4 val = make_uint4(pack_bf16x2(src[0], src[1]), pack_bf16x2(src[2], src[3]),
+                                             pack_bf16x2(src[4], src[5]), pack_bf16x2(src[6], src[7]));
+                __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.C) +
+                                     static_cast<int64_t>(ti.m0 + j0 + i) * p.ldc + ti.wb * 128;
+                reinterpret_cast<uint4*>(dst)[c8] = val;
+              }
+            }
+          }
+        } else {
+          // swiglu: gate = weight rows 0..63, up = rows 64..127 of the block;
+          // h row = 64 bf16 = 8 x 16 B; 16 rows per pass
+#pragma unroll
+          for (int pass = 0; pass < 2; ++pass) {
+            const int i = pass * 16 + (et >> 3);
+            const int c8 = et & 7;
+            if (i < rows) {
+              const float* g = sOut + i * 128 + c8 * 8;
+              const float* u = g + 64;
+              uint32_t pk[4];
+#pragma unroll
+              for (int k2 = 0; k2 < 4; ++k2)
+                pk[k2] = pack_bf16x2(silu(g[2 * k2]) * u[2 * k2], silu(g[2 * k2 + 1]) * u[2 * k2 + 1]);
+              __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.C) +
+                                   static_cast<int64_t>(ti.m0 + j0 + i) * p.ldc + ti.wb * 64;
+              reinterpret_cast<uint4*>(dst)[c8] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+          }
+        }
+        epi_bar();  // sOut is rewritten by the next slab
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
+      if (++acc == NUM_ACC) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+bool encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows,
+                    uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {K, rows};
+  cuuint64_t strides[1] = {K * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int kMode, int TN>
+cudaError_t run_t(const GemmLaunch& L, cudaStream_t stream) {
+  using Cfg = TCfg<kMode, TN>;
+  static bool attr_done[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_t_kernel<kMode, TN>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Cfg::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_done[dev] = true;
+  }
+  const bool grouped = L.group_sizes != nullptr;
+  const int E = grouped ? L.E : 1;
+  CUtensorMap tmW, tmX[kXBoxes];
+  const uint32_t wbox = kMode == kTSwiglu ? 64 : 128;
+  if (!encode_bf16_2d(&tmW, L.B, L.K, static_cast<uint64_t>(E) * L.N, wbox))
+    return cudaErrorInvalidValue;
+  for (int i = 0; i < kXBoxes; ++i)
+    if (!encode_bf16_2d(&tmX[i], L.A, L.K, L.rows, 32u << i)) return cudaErrorInvalidValue;
+  TParams p{};
+  p.M_dense = grouped ? 0 : L.rows;
+  p.N = L.N;
+  p.K = L.K;
+  p.E = E;
+  p.group_sizes = L.group_sizes;
+  p.group_offsets = L.group_offsets;
+  p.rows_total = L.rows;
+  p.C = L.C;
+  p.ldc = kMode == kTSwiglu ? L.N / 2 : L.N;
+  p.out_f32 = L.out_f32;
+  p.status = L.status;
+  const int WB = kMode == kTSwiglu ? (L.N / 2) / 64 : L.N / 128;
+  const long long chunks_ub = grouped ? (static_cast<long long>(L.rows) + TN - 1) / TN + E
+                                      : (static_cast<long long>(L.rows) + TN - 1) / TN;
+  const long long tiles_ub = chunks_ub * WB;
+  const int sms = device_sm_count();
+  const int grid = static_cast<int>(tiles_ub < sms ? (tiles_ub > 0 ? tiles_ub : 1) : sms);
+  grouped_gemm_t_kernel<kMode, TN><<<grid, 192, Cfg::SMEM_BYTES, stream>>>(
+      tmW, tmX[0], tmX[1], tmX[2], tmX[3], p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool grouped_gemm_t_supported(const GemmLaunch& L) {
+  if (L.A_scales != nullptr || L.B_scales != nullptr) return false;
+  if (L.E > 1024) return false;
+  if (L.mode == kModeStore) return L.N % 128 == 0 && L.K % 64 == 0;
+  if (L.mode == kModeSwiglu) return (L.N / 2) % 64 == 0 && L.N % 2 == 0 && L.K % 64 == 0;
+  return false;
+}
+
+cudaError_t launch_grouped_gemm_t(const GemmLaunch& L, cudaStream_t stream) {
+  // Token tile sized to the groups: small groups (decode) keep 64-row token
+  // tiles so 8 stages fit and more weight bytes stay in flight per SM.
+  const bool small = L.group_sizes != nullptr && L.rows <= 64 * L.E;
+  if (L.mode == kModeSwiglu)
+    return small ? run_t<kTSwiglu, 64>(L, stream) : run_t<kTSwiglu, 256>(L, stream);
+  if (L.mode == kModeStore)
+    return small ? run_t<kTStore, 64>(L, stream) : run_t<kTStore, 256>(L, stream);
+  return cudaErrorInvalidValue;
+}
+
+bool grouped_gemm_t_preferred(const GemmLaunch& L) {
+  // measured on B200: weight-row tiles win for the down/store GEMM at every
+  // group size once the token tile fits the groups, and for SwiGLU on small
+  // groups; token-row tiles keep SwiGLU on large groups (their epilogue needs
+  // no shared-memory pairing of gate and up)
+  if (L.mode == kModeStore) return true;
+  return L.group_sizes != nullptr && L.rows <= 64 * L.E;
+}
+
+}  // namespace moe

@@ -12,6 +12,7 @@ enum GemmMode { kModeStore = 0, kModeSwiglu = 1, kModeSwigluFp8 = 2, kModeFp8Sto
 
 struct GemmLaunch {
   int mode = kModeStore;
+  int tiling = 0;  // GemmTiling
   // grouped mode: tables non-null, rows = P; dense mode: tables null, rows = M
   int rows = 0;
   int N = 0;  // rows of B per expert
@@ -33,8 +34,15 @@ struct GemmLaunch {
   int32_t* status = nullptr;
 };
 
+// Tiling of the grouped GEMM: token-row tiles (grouped_gemm.cu) or
+// weight-row tiles with the tokens on the MMA's N side (grouped_gemm_t.cu).
+enum GemmTiling { kTilingAuto = 0, kTilingRows = 1, kTilingWeights = 2 };
+
 // Each returns cudaSuccess or the launch error.
 cudaError_t launch_grouped_gemm(const GemmLaunch& L, cudaStream_t stream);
+cudaError_t launch_grouped_gemm_t(const GemmLaunch& L, cudaStream_t stream);
+bool grouped_gemm_t_supported(const GemmLaunch& L);
+bool grouped_gemm_t_preferred(const GemmLaunch& L);
 
 cudaError_t launch_route_topk(const float* logits, int T, int E, int k, int score_fn,
                               int renormalize, int32_t* ids, float* weights, cudaStream_t stream);

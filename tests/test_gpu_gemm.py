@@ -67,9 +67,13 @@ GEMM_CASES = [
 ]
 
 
+TILINGS = [0x10, 0x20]   # MOE_TILE_TOKEN_ROWS, MOE_TILE_WEIGHT_ROWS
+
+
+@pytest.mark.parametrize("tiling", TILINGS)
 @pytest.mark.parametrize("f32", [False, True])
 @pytest.mark.parametrize("T,E,k,H,F,sizes", GEMM_CASES)
-def test_grouped_gemm_store(T, E, k, H, F, sizes, f32):
+def test_grouped_gemm_store(T, E, k, H, F, sizes, f32, tiling):
     gu = _gu()
     import moe_routed_expert_top_b200 as M
     cfg, ids, hidden, L, tables, status, x_perm, ref, wgu, wd = _setup(T, E, k, H, F, 1, sizes)
@@ -77,7 +81,8 @@ def test_grouped_gemm_store(T, E, k, H, F, sizes, f32):
     C = torch.full((L["P"], 2 * F), float("nan"), dtype=torch.float32 if f32 else torch.bfloat16,
                    device="cuda")
     M.moe_grouped_gemm(prob, 0, 2 * F, H, x_perm, None, wgu, None, tables,
-                       M.MOE_EPI_STORE_F32 if f32 else M.MOE_EPI_STORE, C, None, None, status)
+                       (M.MOE_EPI_STORE_F32 if f32 else M.MOE_EPI_STORE) | tiling, C, None, None,
+                       status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     refC = _oracle_rows_gemm(hidden, wgu, ref, E, k)
@@ -88,15 +93,16 @@ def test_grouped_gemm_store(T, E, k, H, F, sizes, f32):
         gu.assert_within_tol(gu.f64(C), refC, "gate_up store")
 
 
+@pytest.mark.parametrize("tiling", TILINGS)
 @pytest.mark.parametrize("T,E,k,H,F,sizes", GEMM_CASES)
-def test_grouped_gemm_swiglu(T, E, k, H, F, sizes):
+def test_grouped_gemm_swiglu(T, E, k, H, F, sizes, tiling):
     gu = _gu()
     import moe_routed_expert_top_b200 as M
     cfg, ids, hidden, L, tables, status, x_perm, ref, wgu, wd = _setup(T, E, k, H, F, 2, sizes)
     prob = gu.problem(cfg)
     h = torch.full((L["P"], F), float("nan"), dtype=torch.bfloat16, device="cuda")
-    M.moe_grouped_gemm(prob, 0, 2 * F, H, x_perm, None, wgu, None, tables, M.MOE_EPI_SWIGLU, h,
-                       None, None, status)
+    M.moe_grouped_gemm(prob, 0, 2 * F, H, x_perm, None, wgu, None, tables,
+                       M.MOE_EPI_SWIGLU | tiling, h, None, None, status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     G = _oracle_rows_gemm(hidden, wgu, ref, E, k)
@@ -169,8 +175,9 @@ def test_grouped_gemm_fp8_block_scaled(T, E, k, H, F, sizes):
             gu.assert_within_tol(gu.f64(y), refy, "fp8 down")
 
 
+@pytest.mark.parametrize("tiling", TILINGS)
 @pytest.mark.parametrize("M_rows,N,K", [(1, 128, 64), (300, 512, 448), (4096 + 17, 256, 256)])
-def test_dense_gemm_store(M_rows, N, K):
+def test_dense_gemm_store(M_rows, N, K, tiling):
     gu = _gu()
     import moe_routed_expert_top_b200 as M
     g = torch.Generator(device="cuda")
@@ -179,8 +186,8 @@ def test_dense_gemm_store(M_rows, N, K):
     B = (torch.randn(N, K, generator=g, device="cuda") * 0.05).to(torch.bfloat16)
     C = torch.empty(M_rows, N, dtype=torch.bfloat16, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    M.moe_grouped_gemm(None, M_rows, N, K, A, None, B, None, None, M.MOE_EPI_STORE, C, None, None,
-                       status)
+    M.moe_grouped_gemm(None, M_rows, N, K, A, None, B, None, None, M.MOE_EPI_STORE | tiling, C,
+                       None, None, status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     gu.assert_within_tol(gu.f64(C), gu.f64(A) @ gu.f64(B).T, "dense")
