@@ -101,9 +101,9 @@ enum {
  *   MOE_TILE_TOKEN_ROWS  128 token rows x N columns per tile (every epilogue)
  *   MOE_TILE_WEIGHT_ROWS 128 weight rows x (the expert's tokens, <= 256, rounded
  *                        up to 16) per tile: MMA work follows the real group
- *                        sizes; bf16 mode with MOE_EPI_STORE / STORE_F32
- *                        (N % 128 == 0) or MOE_EPI_SWIGLU (N % 128 == 0) only,
- *                        else MOE_ERR_UNSUPPORTED. */
+ *                        sizes; MOE_EPI_STORE / STORE_F32 (N % 128 == 0; in
+ *                        FP8 mode also K <= 4096) or bf16 MOE_EPI_SWIGLU
+ *                        (N % 128 == 0) only, else MOE_ERR_UNSUPPORTED. */
 enum { MOE_TILE_AUTO = 0x00, MOE_TILE_TOKEN_ROWS = 0x10, MOE_TILE_WEIGHT_ROWS = 0x20 };
 
 /* One MoE layer's shape and routing options. */

@@ -39,7 +39,7 @@ namespace moe {
 
 namespace {
 
-enum TMode { kTStore = 0, kTSwiglu = 1 };
+enum TMode { kTStore = 0, kTSwiglu = 1, kTFp8Store = 2 };
 
 constexpr int kXBoxes = 4;  // token-tile TMA boxes of 32, 64, 128, 256 rows
 
@@ -53,7 +53,10 @@ struct TParams {
   int rows_total;
   void* C;
   int ldc;      // output row length in elements
-  int out_f32;  // store mode: fp32 C
+  int out_f32;  // store modes: fp32 C
+  const float* A_scales;  // FP8: activation scales [rows, KBS]
+  const float* B_scales;  // FP8: weight block scales [E, N/128, KBS]
+  int KBS;                // FP8: K / 128
   int32_t* status;
 };
 
@@ -61,19 +64,27 @@ __host__ __device__ constexpr int tmin(int a, int b) { return a < b ? a : b; }
 
 template <int kMode, int TN>
 struct TCfg {
-  static constexpr int BK = 64;           // bf16 elements per 128-byte smem row
-  static constexpr int K_STEPS = 4;       // MMAs (K=16) per stage
+  static constexpr bool kFp8 = kMode == kTFp8Store;
+  static constexpr int BK = kFp8 ? 128 : 64;  // elements per 128-byte smem row
+  static constexpr int K_STEPS = 4;           // MMAs (K = 16 bf16 / 32 e4m3) per stage
   static constexpr int A_BYTES = 128 * 128;     // weight tile: 128 rows x 128 B
   static constexpr int B_BYTES = TN * 128;      // token tile: up to TN rows x 128 B
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = tmin(8, (200 * 1024) / STAGE_BYTES);
-  static constexpr int NUM_ACC = 2;
-  static constexpr int TMEM_COLS = 2 * TN;      // TN <= 256
+  static constexpr int STAGES = tmin(8, ((kFp8 ? 192 : 200) * 1024) / STAGE_BYTES);
+  // FP8: one TMEM buffer per 128-wide K-block, as many in flight as 512 columns
+  // hold (the MMA -> epilogue -> release round trip per K-block is latency
+  // bound); bf16: 2 tile buffers
+  static constexpr int NUM_ACC = kFp8 ? 512 / TN : 2;
+  static constexpr int TMEM_COLS = NUM_ACC * TN;
   static constexpr int STAGE_OUT_BYTES = 32 * 128 * 4;  // 32 token rows x 128 fp32
+  static constexpr int MAX_KBS = 32;                    // FP8: K <= 4096
+  static constexpr int SA_BYTES = kFp8 ? TN * MAX_KBS * 4 : 0;
   static constexpr int NUM_BARS = 2 * STAGES + 2 * NUM_ACC + 1;
   static constexpr int MAX_E = 1024;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STAGE_OUT_BYTES +
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STAGE_OUT_BYTES + SA_BYTES +
                                     NUM_BARS * 8 + 16 + (MAX_E + 8) * 4;
+  static_assert(TMEM_COLS <= 512 && (TMEM_COLS & (TMEM_COLS - 1)) == 0, "tensor memory");
+  static_assert(!kFp8 || TN <= 64, "FP8 keeps TN columns per K-block buffer, 4 buffers");
   static constexpr int WROWS = (kMode == kTSwiglu) ? 64 : 128;  // output columns per tile
   static_assert(TN % 32 == 0 && TN >= 32 && TN <= 256, "token tile");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
@@ -122,6 +133,38 @@ __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: 
 
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
 
+// Write `rows` staged token rows (sOut[i][0..128), fp32) to C rows row0.. at
+// column col0, fp32 or bf16, 16-byte stores; 128 epilogue threads (et).
+__device__ __forceinline__ void store_rows(const TParams& p, const float* sOut, int et, int rows,
+                                           int row0, int col0) {
+  if (p.out_f32) {
+#pragma unroll
+    for (int pass = 0; pass < 8; ++pass) {
+      const int i = pass * 4 + (et >> 5);
+      const int c4 = et & 31;
+      if (i < rows) {
+        const float4 val = reinterpret_cast<const float4*>(sOut + i * 128)[c4];
+        float* dst = static_cast<float*>(p.C) + static_cast<int64_t>(row0 + i) * p.ldc + col0;
+        reinterpret_cast<float4*>(dst)[c4] = val;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int pass = 0; pass < 4; ++pass) {
+      const int i = pass * 8 + (et >> 4);
+      const int c8 = et & 15;
+      if (i < rows) {
+        const float* src = sOut + i * 128 + c8 * 8;
+        const uint4 val = make_uint4(pack_bf16x2(src[0], src[1]), pack_bf16x2(src[2], src[3]),
+                                     pack_bf16x2(src[4], src[5]), pack_bf16x2(src[6], src[7]));
+        __nv_bfloat16* dst =
+            static_cast<__nv_bfloat16*>(p.C) + static_cast<int64_t>(row0 + i) * p.ldc + col0;
+        reinterpret_cast<uint4*>(dst)[c8] = val;
+      }
+    }
+  }
+}
+
 template <int kMode, int TN>
 __global__ void __launch_bounds__(192, 1)
     grouped_gemm_t_kernel(const __grid_constant__ CUtensorMap tmW,
@@ -139,8 +182,9 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* sA = smem;                                   // weight tiles
   uint8_t* sB = smem + STAGES * Cfg::A_BYTES;           // token tiles
   float* sOut = reinterpret_cast<float*>(sB + STAGES * Cfg::B_BYTES);  // [32][128]
+  float* sSa = sOut + 32 * 128;  // FP8: activation scales of the tile's tokens [TN][KBS]
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sOut) +
-                                               Cfg::STAGE_OUT_BYTES);
+                                               Cfg::STAGE_OUT_BYTES + Cfg::SA_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NUM_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   // set only by epilogue threads, read only after their shared barrier: the four
@@ -282,6 +326,35 @@ __global__ void __launch_bounds__(192, 1)
         TTile ti;
         if (!t_decode(p, cpre, E, WB, TN, t, ti)) continue;
         const int nmma = (ti.nt + 15) & ~15;
+        if constexpr (Cfg::kFp8) {
+          // one TMEM buffer per 128-wide K-block: the epilogue scales and sums them
+          const uint32_t idesc8 = idesc_e4m3_f32(128, nmma);
+          for (int kb = 0; kb < KB; ++kb) {
+            if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag, p.status) ||
+                !mbar_wait(full0 + 8 * stage, phase, abort_flag, p.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t d = tmem_base + static_cast<uint32_t>(acc * TN);
+            const uint64_t adesc = smem_desc_sw128(smem_u32(sA + stage * Cfg::A_BYTES));
+            const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + stage * Cfg::B_BYTES));
+#pragma unroll
+            for (int k = 0; k < Cfg::K_STEPS; ++k)
+              mma_fp8(d, adesc + 2 * k, bdesc + 2 * k, idesc8, k != 0 ? 1u : 0u);
+            mma_commit(empty0 + 8 * stage);
+            mma_commit(tfull0 + 8 * acc);
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+            if (++acc == NUM_ACC) {
+              acc = 0;
+              acc_phase ^= 1u;
+            }
+          }
+          continue;
+        }
         const uint32_t idesc = idesc_bf16_f32(128, nmma);
         if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag, p.status)) {
           ok = false;
@@ -327,6 +400,90 @@ __global__ void __launch_bounds__(192, 1)
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
       TTile ti;
       if (!t_decode(p, cpre, E, WB, TN, t, ti)) continue;
+      if constexpr (Cfg::kFp8) {
+        // y[t, w] = sum_kb sw[e, wb, kb] * sa[t, kb] * (Wq_kb Xq_kb^T)[w, t]
+        // stage s[kb][t] = sw[e, wb, kb] * sa[m0 + t, kb], K-block major so each
+        // K-block's column scales are read as 16-byte vectors (same address in
+        // every thread: a broadcast)
+        const int nsa = ti.nt * p.KBS;
+        const float* gsa = p.A_scales + static_cast<int64_t>(ti.m0) * p.KBS;
+        const float* gsw =
+            p.B_scales + (static_cast<int64_t>(ti.e) * (p.N / 128) + ti.wb) * p.KBS;
+        // 8 independent loads in flight per thread per round (at most TN*32/1024 rounds)
+        for (int base = 0; base < nsa; base += 8 * 128) {
+          float a[8], b[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int i = base + j * 128 + et;
+            const bool in = i < nsa;
+            a[j] = in ? __ldg(gsa + i) : 0.0f;
+            b[j] = in ? __ldg(gsw + (i % p.KBS)) : 0.0f;
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int i = base + j * 128 + et;
+            if (i < nsa) {
+              const int tok = i / p.KBS;
+              const int kb = i - tok * p.KBS;
+              sSa[kb * TN + tok] = a[j] * b[j];
+            }
+          }
+        }
+        epi_bar();
+        float accv[TN];
+#pragma unroll
+        for (int i = 0; i < TN; ++i) accv[i] = 0.0f;
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t tbk = lane_base + static_cast<uint32_t>(acc * TN);
+          const float4* s4 = reinterpret_cast<const float4*>(sSa + kb * TN);
+          uint32_t v[TN / 32][32];
+#pragma unroll
+          for (int c = 0; c < TN / 32; ++c)
+            if (c * 32 < ti.nt) tmem_ld32(tbk + c * 32, v[c]);  // uniform across the warp
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < TN / 32; ++c) {
+            if (c * 32 < ti.nt) {
+#pragma unroll
+              for (int i4 = 0; i4 < 8; ++i4) {
+                const float4 s = s4[c * 8 + i4];
+                const int col = c * 32 + i4 * 4;
+                accv[col + 0] = fmaf(s.x, __uint_as_float(v[c][i4 * 4 + 0]), accv[col + 0]);
+                accv[col + 1] = fmaf(s.y, __uint_as_float(v[c][i4 * 4 + 1]), accv[col + 1]);
+                accv[col + 2] = fmaf(s.z, __uint_as_float(v[c][i4 * 4 + 2]), accv[col + 2]);
+                accv[col + 3] = fmaf(s.w, __uint_as_float(v[c][i4 * 4 + 3]), accv[col + 3]);
+              }
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
+          if (++acc == NUM_ACC) {
+            acc = 0;
+            acc_phase ^= 1u;
+          }
+        }
+        if (!ok) *epi_abort = 1;
+        epi_bar();
+        if (*epi_abort) break;
+#pragma unroll
+        for (int c = 0; c < TN / 32; ++c) {
+          if (c * 32 < ti.nt) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sOut[i * 128 + r] = accv[c * 32 + i];
+            epi_bar();
+            store_rows(p, sOut, et, tmin(32, ti.nt - c * 32), ti.m0 + c * 32, ti.wb * 128);
+            epi_bar();
+          }
+        }
+        continue;
+      }
       if (!mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, p.status)) *epi_abort = 1;
       epi_bar();  // every epilogue warp arrives here whether its wait succeeded or not
       if (*epi_abort) break;
@@ -425,17 +582,21 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-bool encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows,
-                    uint32_t box_rows) {
+// K-major [rows, K] tensor of bf16 (or e4m3 bytes), boxes of 128 bytes x box_rows,
+// 128-byte swizzle, zero fill out of bounds.
+bool encode_kmajor_2d(CUtensorMap* map, const void* base, bool fp8, uint64_t K, uint64_t rows,
+                      uint32_t box_rows) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
+  const uint32_t elt = fp8 ? 1 : 2;
   cuuint64_t dims[2] = {K, rows};
-  cuuint64_t strides[1] = {K * 2};
-  cuuint32_t box[2] = {64, box_rows};
+  cuuint64_t strides[1] = {K * elt};
+  cuuint32_t box[2] = {128 / elt, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+            const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int kMode, int TN>
@@ -455,10 +616,11 @@ cudaError_t run_t(const GemmLaunch& L, cudaStream_t stream) {
   const int E = grouped ? L.E : 1;
   CUtensorMap tmW, tmX[kXBoxes];
   const uint32_t wbox = kMode == kTSwiglu ? 64 : 128;
-  if (!encode_bf16_2d(&tmW, L.B, L.K, static_cast<uint64_t>(E) * L.N, wbox))
+  if (!encode_kmajor_2d(&tmW, L.B, Cfg::kFp8, L.K, static_cast<uint64_t>(E) * L.N, wbox))
     return cudaErrorInvalidValue;
   for (int i = 0; i < kXBoxes; ++i)
-    if (!encode_bf16_2d(&tmX[i], L.A, L.K, L.rows, 32u << i)) return cudaErrorInvalidValue;
+    if (!encode_kmajor_2d(&tmX[i], L.A, Cfg::kFp8, L.K, L.rows, 32u << i))
+      return cudaErrorInvalidValue;
   TParams p{};
   p.M_dense = grouped ? 0 : L.rows;
   p.N = L.N;
@@ -470,6 +632,9 @@ cudaError_t run_t(const GemmLaunch& L, cudaStream_t stream) {
   p.C = L.C;
   p.ldc = kMode == kTSwiglu ? L.N / 2 : L.N;
   p.out_f32 = L.out_f32;
+  p.A_scales = L.A_scales;
+  p.B_scales = L.B_scales;
+  p.KBS = L.K / 128;
   p.status = L.status;
   const int WB = kMode == kTSwiglu ? (L.N / 2) / 64 : L.N / 128;
   const long long chunks_ub = grouped ? (static_cast<long long>(L.rows) + TN - 1) / TN + E
@@ -485,8 +650,11 @@ cudaError_t run_t(const GemmLaunch& L, cudaStream_t stream) {
 }  // namespace
 
 bool grouped_gemm_t_supported(const GemmLaunch& L) {
-  if (L.A_scales != nullptr || L.B_scales != nullptr) return false;
   if (L.E > 1024) return false;
+  if (L.mode == kModeFp8Store)
+    return L.A_scales != nullptr && L.B_scales != nullptr && L.N % 128 == 0 &&
+           L.K % 128 == 0 && L.K <= 128 * 32;
+  if (L.A_scales != nullptr || L.B_scales != nullptr) return false;
   if (L.mode == kModeStore) return L.N % 128 == 0 && L.K % 64 == 0;
   if (L.mode == kModeSwiglu) return (L.N / 2) % 64 == 0 && L.N % 2 == 0 && L.K % 64 == 0;
   return false;
@@ -500,6 +668,7 @@ cudaError_t launch_grouped_gemm_t(const GemmLaunch& L, cudaStream_t stream) {
     return small ? run_t<kTSwiglu, 64>(L, stream) : run_t<kTSwiglu, 256>(L, stream);
   if (L.mode == kModeStore)
     return small ? run_t<kTStore, 64>(L, stream) : run_t<kTStore, 256>(L, stream);
+  if (L.mode == kModeFp8Store) return run_t<kTFp8Store, 64>(L, stream);
   return cudaErrorInvalidValue;
 }
 
@@ -508,7 +677,7 @@ bool grouped_gemm_t_preferred(const GemmLaunch& L) {
   // group size once the token tile fits the groups, and for SwiGLU on small
   // groups; token-row tiles keep SwiGLU on large groups (their epilogue needs
   // no shared-memory pairing of gate and up)
-  if (L.mode == kModeStore) return true;
+  if (L.mode == kModeStore || L.mode == kModeFp8Store) return true;
   return L.group_sizes != nullptr && L.rows <= 64 * L.E;
 }
 

@@ -144,7 +144,8 @@ def test_grouped_gemm_swiglu_fp8_epilogue(T, E, k, H, F, sizes):
 
 @pytest.mark.parametrize("T,E,k,H,F,sizes", [(200, 8, 2, 256, 384, None),
                                             (260, 8, 3, 512, 256, [0, 1, 127, 128, 129, 0, 255, 140])])
-def test_grouped_gemm_fp8_block_scaled(T, E, k, H, F, sizes):
+@pytest.mark.parametrize("tiling", TILINGS)
+def test_grouped_gemm_fp8_block_scaled(T, E, k, H, F, sizes, tiling):
     gu = _gu()
     import moe_routed_expert_top_b200 as M
     cfg, ids, hidden, L, tables, status, x_perm, ref, wgu, wd = _setup(T, E, k, H, F, 4, sizes)
@@ -166,7 +167,8 @@ def test_grouped_gemm_fp8_block_scaled(T, E, k, H, F, sizes):
                        device="cuda")
         M.moe_grouped_gemm(prob, 0, H, F, torch.from_numpy(qa).cuda(), torch.from_numpy(sa).cuda(),
                            torch.from_numpy(wq).cuda(), torch.from_numpy(ws).cuda(), tables,
-                           M.MOE_EPI_STORE_F32 if f32 else M.MOE_EPI_STORE, y, None, None, status)
+                           (M.MOE_EPI_STORE_F32 if f32 else M.MOE_EPI_STORE) | tiling, y, None,
+                           None, status)
         torch.cuda.synchronize()
         assert int(status.item()) == 0
         if f32:
