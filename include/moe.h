@@ -97,14 +97,29 @@ enum {
 
 /* Tiling choice, OR-ed into moe_grouped_gemm's `epilogue` argument. Both
  * compute the same result.
- *   MOE_TILE_AUTO        the library's choice (weight rows where supported)
+ *   MOE_TILE_AUTO        the library's choice: weight-row pairs for bf16 problems
+ *                        whose experts average more than 64 rows (and dense
+ *                        problems), else weight rows where supported, else
+ *                        token rows
  *   MOE_TILE_TOKEN_ROWS  128 token rows x N columns per tile (every epilogue)
  *   MOE_TILE_WEIGHT_ROWS 128 weight rows x (the expert's tokens, <= 256, rounded
  *                        up to 16) per tile: MMA work follows the real group
  *                        sizes; MOE_EPI_STORE / STORE_F32 (N % 128 == 0; in
  *                        FP8 mode also K <= 4096) or bf16 MOE_EPI_SWIGLU
- *                        (N % 128 == 0) only, else MOE_ERR_UNSUPPORTED. */
-enum { MOE_TILE_AUTO = 0x00, MOE_TILE_TOKEN_ROWS = 0x10, MOE_TILE_WEIGHT_ROWS = 0x20 };
+ *                        (N % 128 == 0) only, else MOE_ERR_UNSUPPORTED.
+ *   MOE_TILE_WEIGHT_ROWS_PAIR  256 weight rows x (tokens, <= 256) per tile,
+ *                        computed by two CTAs of a cluster with one 256-row
+ *                        MMA (each CTA fetches half of the weight rows and half
+ *                        of the token rows); bf16 only: MOE_EPI_STORE /
+ *                        STORE_F32 (N % 256 == 0) or MOE_EPI_SWIGLU
+ *                        (N % 256 == 0), K % 64 == 0, E <= 1024, else
+ *                        MOE_ERR_UNSUPPORTED. */
+enum {
+  MOE_TILE_AUTO = 0x00,
+  MOE_TILE_TOKEN_ROWS = 0x10,
+  MOE_TILE_WEIGHT_ROWS = 0x20,
+  MOE_TILE_WEIGHT_ROWS_PAIR = 0x30
+};
 
 /* One MoE layer's shape and routing options. */
 typedef struct moe_problem {

@@ -19,8 +19,8 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmoe_b200.so")
 
-SOURCES = ["api.cu", "grouped_gemm.cu", "grouped_gemm_t.cu", "route_permute.cu", "tables.cu",
-           "elementwise.cu", "no_alloc.cu"]
+SOURCES = ["api.cu", "grouped_gemm.cu", "grouped_gemm_t.cu", "grouped_gemm_t2.cu",
+           "route_permute.cu", "tables.cu", "elementwise.cu", "no_alloc.cu"]
 # translation units whose float32 results must not depend on FMA contraction
 NO_FMA = {"route_permute.cu", "elementwise.cu"}
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -176,7 +176,7 @@ moe_status moe_grouped_gemm(const moe_problem* prob, int32_t M_rows, int32_t N, 
   moe::GemmLaunch g;
   const int tiling = (epilogue >> 4) & 0xF;
   epilogue &= 0xF;
-  if (tiling > moe::kTilingWeights) return MOE_ERR_INVALID_ARG;
+  if (tiling > moe::kTilingWeightsPair) return MOE_ERR_INVALID_ARG;
   g.tiling = tiling;
   if (tables != nullptr) {
     moe_status s = check_problem(prob, false);
@@ -236,6 +236,8 @@ moe_status moe_grouped_gemm(const moe_problem* prob, int32_t M_rows, int32_t N, 
   g.debug_h = debug_h;
   g.status = dev_status;
   if (g.tiling == moe::kTilingWeights && !moe::grouped_gemm_t_supported(g))
+    return MOE_ERR_UNSUPPORTED;
+  if (g.tiling == moe::kTilingWeightsPair && !moe::grouped_gemm_pair_supported(g))
     return MOE_ERR_UNSUPPORTED;
   MOE_CUDA_TRY(moe::launch_grouped_gemm(g, reinterpret_cast<cudaStream_t>(stream)));
   return MOE_OK;

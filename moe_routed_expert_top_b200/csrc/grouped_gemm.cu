@@ -373,12 +373,18 @@ __global__ void __launch_bounds__(192, 1)
         } else if constexpr (kMode == kModeSwiglu) {
           constexpr int HN = BN / 2;
           __nv_bfloat16* C = static_cast<__nv_bfloat16*>(p.C);
+          uint32_t g[32], u[32], gn[32], un[32];
+          tmem_ld32(tb, g);
+          tmem_ld32(tb + HN, u);
+          tmem_ld_wait();
 #pragma unroll 1
           for (int c = 0; c < HN / 32; ++c) {
-            uint32_t g[32], u[32];
-            tmem_ld32(tb + c * 32, g);
-            tmem_ld32(tb + HN + c * 32, u);
-            tmem_ld_wait();
+            // the next chunk's TMEM loads run while this chunk is computed and stored
+            const bool more = c + 1 < HN / 32;
+            if (more) {
+              tmem_ld32(tb + (c + 1) * 32, gn);
+              tmem_ld32(tb + HN + (c + 1) * 32, un);
+            }
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -392,6 +398,14 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
               for (int i = 0; i < 4; ++i)
                 dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            }
+            if (more) {
+              tmem_ld_wait();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                g[i] = gn[i];
+                u[i] = un[i];
+              }
             }
           }
         } else {  // kModeSwigluFp8: 128 h columns = one 1x128 quantisation tile
@@ -619,6 +633,9 @@ static cudaError_t run_gemm(const GemmLaunch& L, cudaStream_t stream) {
 }
 
 cudaError_t launch_grouped_gemm(const GemmLaunch& L, cudaStream_t stream) {
+  if (L.tiling == kTilingWeightsPair || (L.tiling == kTilingAuto && grouped_gemm_pair_preferred(L)))
+    return grouped_gemm_pair_supported(L) ? launch_grouped_gemm_pair(L, stream)
+                                          : cudaErrorNotSupported;
   if (grouped_gemm_t_supported(L) &&
       (L.tiling == kTilingWeights || (L.tiling == kTilingAuto && grouped_gemm_t_preferred(L))))
     return launch_grouped_gemm_t(L, stream);

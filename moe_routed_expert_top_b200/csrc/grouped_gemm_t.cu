@@ -92,6 +92,7 @@ struct TCfg {
 
 struct TTile {
   int e, wb, m0, nt;
+  int chunks;  // token tiles of this expert (tiles that read the same weights)
 };
 
 // Tile t -> (expert, weight block, token chunk). cpre[e] = token chunks of the
@@ -116,6 +117,7 @@ __device__ __forceinline__ bool t_decode(const TParams& p, const int* cpre, int 
   const int off = p.group_offsets ? __ldg(p.group_offsets + e) : 0;
   ti.e = e;
   ti.wb = wb;
+  ti.chunks = chunks;
   ti.m0 = off + c * TN;
   ti.nt = tmin(TN, size - c * TN);
   if (ti.nt <= 0 || ti.m0 < 0 || ti.m0 + ti.nt > p.rows_total) {
@@ -265,7 +267,8 @@ __global__ void __launch_bounds__(192, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const uint64_t pol_act = l2_policy_evict_last();
-      const uint64_t pol_w = l2_policy_evict_first();
+      const uint64_t pol_w1 = l2_policy_by_code(MOE_W_POLICY_SINGLE);
+      const uint64_t pol_wn = l2_policy_by_code(MOE_W_POLICY_MULTI);
       const CUtensorMap* xmaps[kXBoxes] = {&tmX0, &tmX1, &tmX2, &tmX3};
       int stage = 0;
       uint32_t phase = 0;
@@ -278,6 +281,7 @@ __global__ void __launch_bounds__(192, 1)
         const int xb = xbox_for(nmma);
         const uint32_t bytes = Cfg::A_BYTES + (32u << xb) * 128u;
         const int wrow = ti.e * p.N + ti.wb * Cfg::WROWS;
+        const uint64_t pol_w = ti.chunks > 1 ? pol_wn : pol_w1;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.status)) {
             ok = false;
@@ -489,10 +493,13 @@ __global__ void __launch_bounds__(192, 1)
       if (*epi_abort) break;
       tc_fence_after();
       const uint32_t tb = lane_base + static_cast<uint32_t>(acc * TN);
+      uint32_t v[32], vn[32];
+      tmem_ld32(tb, v);
+      tmem_ld_wait();
       for (int j0 = 0; j0 < ti.nt; j0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(tb + j0, v);
-        tmem_ld_wait();
+        // the next slab's TMEM load runs while this slab is staged and stored
+        const bool more = j0 + 32 < ti.nt;
+        if (more) tmem_ld32(tb + j0 + 32, vn);
         // sOut[i][r] = D[r][j0 + i]: token row i, weight row r
 #pragma unroll
         for (int i = 0; i < 32; ++i) sOut[i * 128 + r] = __uint_as_float(v[i]);
@@ -549,6 +556,11 @@ __global__ void __launch_bounds__(192, 1)
           }
         }
         epi_bar();  // sOut is rewritten by the next slab
+        if (more) {
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = vn[i];
+        }
       }
       tc_fence_before();
       __syncwarp();

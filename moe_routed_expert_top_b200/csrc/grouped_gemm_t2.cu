@@ -1,0 +1,538 @@
+// grouped_gemm_t2.cu - weight-row tiles computed by a pair of CTAs (a cluster
+// of two on one TPC) with cta_group::2 MMAs.
+//
+// Same operation and tile order as grouped_gemm_t.cu (TileOPs PR #1580
+// "Grouped-GEMM TMA OOB zero-fill + unpermute out=", Grouped-GEMM kernel:
+// C[e] = A[e] @ B[e]^T over each expert's rows): a pair tile is 256 weight rows
+// x up to TN tokens of one expert. Each CTA of the pair loads its own 128
+// weight rows and its own half of the token rows (no multicast: every CTA
+// fetches its own tiles); the leader CTA issues the M=256 MMA, which reads both
+// CTAs' shared memory and leaves each CTA's 128 rows x N columns in that CTA's
+// tensor memory. Per CTA and per 64-wide K step this moves 16 KB of weights +
+// TN/2 token rows instead of 16 KB + TN rows, for the same MMA work.
+//
+// Pair protocol:
+//   * both CTAs' TMA loads complete on the leader's `full` barrier (the leader
+//     alone arms it with the bytes of both halves);
+//   * the leader's MMA commits to `empty` and `tfull` in both CTAs (multicast
+//     commit), so each producer and each epilogue waits on local barriers;
+//   * both CTAs' epilogue warps release an accumulator on the leader's `tempty`
+//     barrier (8 arrivals);
+//   * a cluster barrier after barrier initialisation and another before tensor
+//     memory is freed keep either CTA from touching the other's shared memory
+//     outside the kernel's lifetime.
+// Modes: store (fp32 or bf16 C) and SwiGLU (64 gate rows stacked over the
+// matching 64 up rows in each CTA's half; TileOPs PR #778, Design; XTuner
+// PR #2089, SiLU(gate)*up). Every wait is bounded (4 s) and sets
+// MOE_DEV_TIMEOUT on expiry.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace moe {
+
+namespace {
+
+enum PMode { kPStore = 0, kPSwiglu = 1 };
+
+constexpr int kPXBoxes = 4;  // boxes of 16, 32, 64, 128 rows for a CTA's half of the tokens
+
+struct PParams {
+  int M_dense;
+  int N;  // rows of W per expert
+  int K;
+  int E;
+  const int32_t* group_sizes;
+  const int32_t* group_offsets;
+  int rows_total;
+  void* C;
+  int ldc;
+  int out_f32;
+  int32_t* status;
+};
+
+__host__ __device__ constexpr int pmin(int a, int b) { return a < b ? a : b; }
+
+template <int kMode, int TN>
+struct PCfg {
+  static constexpr int BK = 64;
+  static constexpr int K_STEPS = 4;
+  static constexpr int A_BYTES = 128 * 128;       // this CTA's 128 weight rows
+  static constexpr int B_BYTES = (TN / 2) * 128;  // this CTA's half of the token rows
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = pmin(8, (200 * 1024) / STAGE_BYTES);
+  static constexpr int NUM_ACC = 2;
+  static constexpr int TMEM_COLS = 2 * TN;
+  static constexpr int STAGE_OUT_BYTES = 32 * 128 * 4;
+  static constexpr int NUM_BARS = 2 * STAGES + 2 * NUM_ACC + 1;
+  static constexpr int MAX_E = 1024;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STAGE_OUT_BYTES +
+                                    NUM_BARS * 8 + 16 + (MAX_E + 8) * 4;
+  static constexpr int PAIR_COLS = (kMode == kPSwiglu) ? 128 : 256;  // output columns per pair tile
+  static constexpr int CTA_COLS = PAIR_COLS / 2;
+  static_assert(TN % 32 == 0 && TN >= 32 && TN <= 256, "token tile");
+  static_assert(TMEM_COLS <= 512, "tensor memory");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+};
+
+struct PTile {
+  int e, wb, m0, nt;
+  int chunks;  // token tiles of this expert (tiles that read the same weights)
+};
+
+__device__ __forceinline__ bool p_decode(const PParams& p, const int* cpre, int E, int WB, int TN,
+                                         int t, PTile& ti) {
+  int lo = 0, hi = E - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (WB * cpre[mid] <= t)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  const int e = lo;
+  const int chunks = cpre[e + 1] - cpre[e];
+  if (chunks <= 0) return false;
+  const int local = t - WB * cpre[e];
+  const int wb = local / chunks;
+  const int c = local - wb * chunks;
+  const int size = p.group_sizes ? __ldg(p.group_sizes + e) : p.M_dense;
+  const int off = p.group_offsets ? __ldg(p.group_offsets + e) : 0;
+  ti.e = e;
+  ti.wb = wb;
+  ti.chunks = chunks;
+  ti.m0 = off + c * TN;
+  ti.nt = pmin(TN, size - c * TN);
+  if (ti.nt <= 0 || ti.m0 < 0 || ti.m0 + ti.nt > p.rows_total) {
+    if (threadIdx.x == 0 && ti.nt > 0) atomicOr(p.status, MOE_DEV_BAD_TABLES_FLAG);
+    return false;
+  }
+  return true;
+}
+
+__device__ __forceinline__ int half_box(int half) {  // smallest of 16/32/64/128 rows >= half
+  return half <= 16 ? 0 : half <= 32 ? 1 : half <= 64 ? 2 : 3;
+}
+
+__device__ __forceinline__ void pepi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ float psilu(float g) { return g / (1.0f + expf(-g)); }
+
+__device__ __forceinline__ void pair_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+
+template <int kMode, int TN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmW,
+                             const __grid_constant__ CUtensorMap tmX0,
+                             const __grid_constant__ CUtensorMap tmX1,
+                             const __grid_constant__ CUtensorMap tmX2,
+                             const __grid_constant__ CUtensorMap tmX3, const PParams p) {
+  using Cfg = PCfg<kMode, TN>;
+  constexpr int STAGES = Cfg::STAGES;
+  constexpr int NUM_ACC = Cfg::NUM_ACC;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * Cfg::A_BYTES;
+  float* sOut = reinterpret_cast<float*>(sB + STAGES * Cfg::B_BYTES);
+  uint64_t* bars =
+      reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sOut) + Cfg::STAGE_OUT_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NUM_BARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* epi_abort = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  int* cpre = reinterpret_cast<int*>(tmem_slot + 4);
+
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = full0 + 8 * STAGES;
+  const uint32_t tfull0 = empty0 + 8 * STAGES;
+  const uint32_t tempty0 = tfull0 + 8 * NUM_ACC;
+  const uint32_t drain_bar = tempty0 + 8 * NUM_ACC;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int E = p.group_sizes ? p.E : 1;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int a = 0; a < NUM_ACC; ++a) {
+      mbar_init(tfull0 + 8 * a, 1);
+      mbar_init(tempty0 + 8 * a, 8);  // 4 epilogue warps in each CTA of the pair
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    *epi_abort = 0;
+    mbar_fence_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmX0);
+    tma_prefetch_desc(&tmX1);
+    tma_prefetch_desc(&tmX2);
+    tma_prefetch_desc(&tmX3);
+  }
+  if (warp == 1) tmem_alloc_pair(smem_u32(tmem_slot), Cfg::TMEM_COLS);
+  {
+    const int per = (E + 191) / 192;
+    const int beg = threadIdx.x * per;
+    int local = 0;
+    for (int i = 0; i < per && beg + i < E; ++i) {
+      const int s = p.group_sizes ? __ldg(p.group_sizes + beg + i) : p.M_dense;
+      local += (s + TN - 1) / TN;
+    }
+    int inc = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, inc, off);
+      if (lane >= off) inc += o;
+    }
+    int* wsum = reinterpret_cast<int*>(sOut);
+    if (lane == 31) wsum[warp] = inc;
+    __syncthreads();
+    int before = 0;
+    for (int w = 0; w < warp; ++w) before += wsum[w];
+    int run = before + inc - local;
+    for (int i = 0; i < per && beg + i < E; ++i) {
+      cpre[beg + i] = run;
+      const int s = p.group_sizes ? __ldg(p.group_sizes + beg + i) : p.M_dense;
+      run += (s + TN - 1) / TN;
+    }
+    if (threadIdx.x == 191) cpre[E] = before + inc;
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any cross-CTA arrive or load completion
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int WB = (kMode == kPSwiglu) ? (p.N / 2) / 128 : p.N / 256;
+  const int total_tiles = WB * cpre[E];
+  const int KB = p.K / Cfg::BK;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      const uint64_t pol_act = l2_policy_evict_last();
+      const uint64_t pol_w1 = l2_policy_by_code(MOE_W_POLICY_SINGLE);
+      const uint64_t pol_wn = l2_policy_by_code(MOE_W_POLICY_MULTI);
+      const CUtensorMap* xmaps[kPXBoxes] = {&tmX0, &tmX1, &tmX2, &tmX3};
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = pair; ok && t < total_tiles; t += npairs) {
+        PTile ti;
+        if (!p_decode(p, cpre, E, WB, TN, t, ti)) continue;
+        const int nmma = (ti.nt + 31) & ~31;
+        const int half = nmma / 2;
+        const int xb = half_box(half);
+        const uint32_t bytes_pair = 2u * (Cfg::A_BYTES + (16u << xb) * 128u);
+        const int wrow = ti.e * p.N + ti.wb * Cfg::PAIR_COLS +
+                         static_cast<int>(rank) * (kMode == kPSwiglu ? 64 : 128);
+        const uint64_t pol_w = ti.chunks > 1 ? pol_wn : pol_w1;
+        const int trow = ti.m0 + static_cast<int>(rank) * half;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb_local = full0 + 8 * stage;
+          const uint32_t fb = cluster_map_shared(fb_local, 0);
+          if (leader) mbar_arrive_expect_tx(fb_local, bytes_pair);
+          const uint32_t a_dst = smem_u32(sA + stage * Cfg::A_BYTES);
+          if constexpr (kMode == kPSwiglu) {
+            tma_load_2d_pair(a_dst, &tmW, kb * Cfg::BK, wrow, fb, pol_w);
+            tma_load_2d_pair(a_dst + 64 * 128, &tmW, kb * Cfg::BK, wrow + p.N / 2, fb, pol_w);
+          } else {
+            tma_load_2d_pair(a_dst, &tmW, kb * Cfg::BK, wrow, fb, pol_w);
+          }
+          tma_load_2d_pair(smem_u32(sB + stage * Cfg::B_BYTES), xmaps[xb], kb * Cfg::BK, trow, fb,
+                           pol_act);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // every load this CTA issued has been consumed (its stage released) before leaving
+      if (ok) {
+        for (int i = 0; i < STAGES; ++i) {
+          mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.status);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader only)
+    if (lane == 0 && leader) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = pair; ok && t < total_tiles; t += npairs) {
+        PTile ti;
+        if (!p_decode(p, cpre, E, WB, TN, t, ti)) continue;
+        const int nmma = (ti.nt + 31) & ~31;
+        const uint32_t idesc = idesc_bf16_f32(256, nmma);
+        if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + static_cast<uint32_t>(acc * TN);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t adesc = smem_desc_sw128(smem_u32(sA + stage * Cfg::A_BYTES));
+          const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + stage * Cfg::B_BYTES));
+#pragma unroll
+          for (int k = 0; k < Cfg::K_STEPS; ++k)
+            mma_bf16_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          mma_commit_pair_mc(empty0 + 8 * stage, 0x3);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit_pair_mc(tfull0 + 8 * acc, 0x3);
+        if (++acc == NUM_ACC) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      pair_commit(drain_bar);
+      mbar_wait_drain(drain_bar, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const int et = threadIdx.x - 64;
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = pair; t < total_tiles; t += npairs) {
+      PTile ti;
+      if (!p_decode(p, cpre, E, WB, TN, t, ti)) continue;
+      if (!mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, p.status)) *epi_abort = 1;
+      pepi_bar();
+      if (*epi_abort) break;
+      tc_fence_after();
+      const uint32_t tb = lane_base + static_cast<uint32_t>(acc * TN);
+      const int col0 = ti.wb * Cfg::PAIR_COLS + static_cast<int>(rank) * Cfg::CTA_COLS;
+      uint32_t v[32], vn[32];
+      tmem_ld32(tb, v);
+      tmem_ld_wait();
+      for (int j0 = 0; j0 < ti.nt; j0 += 32) {
+        const bool more = j0 + 32 < ti.nt;
+        if (more) tmem_ld32(tb + j0 + 32, vn);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sOut[i * 128 + r] = __uint_as_float(v[i]);
+        pepi_bar();
+        const int rows = pmin(32, ti.nt - j0);
+        if constexpr (kMode == kPStore) {
+          if (p.out_f32) {
+#pragma unroll
+            for (int pass = 0; pass < 8; ++pass) {
+              const int i = pass * 4 + (et >> 5);
+              const int c4 = et & 31;
+              if (i < rows) {
+                const float4 val = reinterpret_cast<const float4*>(sOut + i * 128)[c4];
+                float* dst = static_cast<float*>(p.C) +
+                             static_cast<int64_t>(ti.m0 + j0 + i) * p.ldc + col0;
+                reinterpret_cast<float4*>(dst)[c4] = val;
+              }
+            }
+          } else {
+#pragma unroll
+            for (int pass = 0; pass < 4; ++pass) {
+              const int i = pass * 8 + (et >> 4);
+              const int c8 = et & 15;
+              if (i < rows) {
+                const float* src = sOut + i * 128 + c8 * 8;
+                const uint4 val =
+                    make_uint4(pack_bf16x2(src[0], src[1]), pack_bf16x2(src[2], src[3]),
+                               pack_bf16x2(src[4], src[5]), pack_bf16x2(src[6], src[7]));
+                __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.C) +
+                                     static_cast<int64_t>(ti.m0 + j0 + i) * p.ldc + col0;
+                reinterpret_cast<uint4*>(dst)[c8] = val;
+              }
+            }
+          }
+        } else {
+#pragma unroll
+          for (int pass = 0; pass < 2; ++pass) {
+            const int i = pass * 16 + (et >> 3);
+            const int c8 = et & 7;
+            if (i < rows) {
+              const float* g = sOut + i * 128 + c8 * 8;
+              const float* u = g + 64;
+              uint32_t pk[4];
+#pragma unroll
+              for (int k2 = 0; k2 < 4; ++k2)
+                pk[k2] = pack_bf16x2(psilu(g[2 * k2]) * u[2 * k2],
+                                     psilu(g[2 * k2 + 1]) * u[2 * k2 + 1]);
+              __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.C) +
+                                   static_cast<int64_t>(ti.m0 + j0 + i) * p.ldc + col0;
+              reinterpret_cast<uint4*>(dst)[c8] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+          }
+        }
+        pepi_bar();
+        if (more) {
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = vn[i];
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(cluster_map_shared(tempty0 + 8 * acc, 0));
+      if (++acc == NUM_ACC) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  __syncthreads();
+  cluster_sync();  // neither CTA frees tensor memory or exits while its pair still runs
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 p_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+bool p_encode(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows, uint32_t box_rows) {
+  auto fn = p_encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {K, rows};
+  cuuint64_t strides[1] = {K * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int kMode, int TN>
+cudaError_t run_pair(const GemmLaunch& L, cudaStream_t stream) {
+  using Cfg = PCfg<kMode, TN>;
+  static int max_pairs_cache[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (max_pairs_cache[dev] == 0) {
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_pair_kernel<kMode, TN>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Cfg::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    // pairs that can be resident at once (a pair needs both SMs of one TPC free)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(device_sm_count() & ~1));
+    cfg.blockDim = dim3(192);
+    cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, grouped_gemm_pair_kernel<kMode, TN>, &cfg);
+    if (e != cudaSuccess) return e;
+    max_pairs_cache[dev] = n > 0 ? n : 1;
+  }
+  const bool grouped = L.group_sizes != nullptr;
+  const int E = grouped ? L.E : 1;
+  CUtensorMap tmW, tmX[kPXBoxes];
+  if (!p_encode(&tmW, L.B, L.K, static_cast<uint64_t>(E) * L.N, kMode == kPSwiglu ? 64 : 128))
+    return cudaErrorInvalidValue;
+  for (int i = 0; i < kPXBoxes; ++i)
+    if (!p_encode(&tmX[i], L.A, L.K, L.rows, 16u << i)) return cudaErrorInvalidValue;
+  PParams p{};
+  p.M_dense = grouped ? 0 : L.rows;
+  p.N = L.N;
+  p.K = L.K;
+  p.E = E;
+  p.group_sizes = L.group_sizes;
+  p.group_offsets = L.group_offsets;
+  p.rows_total = L.rows;
+  p.C = L.C;
+  p.ldc = kMode == kPSwiglu ? L.N / 2 : L.N;
+  p.out_f32 = L.out_f32;
+  p.status = L.status;
+  const int WB = kMode == kPSwiglu ? (L.N / 2) / 128 : L.N / 256;
+  const long long chunks_ub = grouped ? (static_cast<long long>(L.rows) + TN - 1) / TN + E
+                                      : (static_cast<long long>(L.rows) + TN - 1) / TN;
+  const long long pairs_ub = chunks_ub * WB;
+  const int max_pairs = max_pairs_cache[dev];
+  const int pairs = static_cast<int>(pairs_ub < max_pairs ? (pairs_ub > 0 ? pairs_ub : 1) : max_pairs);
+  grouped_gemm_pair_kernel<kMode, TN><<<2 * pairs, 192, Cfg::SMEM_BYTES, stream>>>(
+      tmW, tmX[0], tmX[1], tmX[2], tmX[3], p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool grouped_gemm_pair_supported(const GemmLaunch& L) {
+  if (L.A_scales != nullptr || L.B_scales != nullptr || L.E > 1024) return false;
+  if (L.mode == kModeStore) return L.N % 256 == 0 && L.K % 64 == 0;
+  if (L.mode == kModeSwiglu) return (L.N / 2) % 128 == 0 && L.K % 64 == 0;
+  return false;
+}
+
+// Measured on B200 with the bf16 workloads (interleaved runs): pairs beat the
+// single-CTA weight-row and token-row tilings once experts hold more than 64
+// rows on average (prefill; down projection by 10-30%), and are on par or
+// slightly behind below that (decode), where the single-CTA kernel's 64-token
+// tiles fit the groups better.
+bool grouped_gemm_pair_preferred(const GemmLaunch& L) {
+  if (!grouped_gemm_pair_supported(L)) return false;
+  return L.group_sizes == nullptr || L.rows > 64 * L.E;
+}
+
+cudaError_t launch_grouped_gemm_pair(const GemmLaunch& L, cudaStream_t stream) {
+  const bool small = L.group_sizes != nullptr && L.rows <= 64 * L.E;
+  if (L.mode == kModeSwiglu)
+    return small ? run_pair<kPSwiglu, 64>(L, stream) : run_pair<kPSwiglu, 256>(L, stream);
+  if (L.mode == kModeStore)
+    return small ? run_pair<kPStore, 64>(L, stream) : run_pair<kPStore, 256>(L, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace moe

@@ -34,15 +34,19 @@ struct GemmLaunch {
   int32_t* status = nullptr;
 };
 
-// Tiling of the grouped GEMM: token-row tiles (grouped_gemm.cu) or
-// weight-row tiles with the tokens on the MMA's N side (grouped_gemm_t.cu).
-enum GemmTiling { kTilingAuto = 0, kTilingRows = 1, kTilingWeights = 2 };
+// Tiling of the grouped GEMM: token-row tiles (grouped_gemm.cu), weight-row
+// tiles with the tokens on the MMA's N side (grouped_gemm_t.cu), or the same
+// weight-row tiles computed by CTA pairs with 256-row MMAs (grouped_gemm_t2.cu).
+enum GemmTiling { kTilingAuto = 0, kTilingRows = 1, kTilingWeights = 2, kTilingWeightsPair = 3 };
 
 // Each returns cudaSuccess or the launch error.
 cudaError_t launch_grouped_gemm(const GemmLaunch& L, cudaStream_t stream);
 cudaError_t launch_grouped_gemm_t(const GemmLaunch& L, cudaStream_t stream);
 bool grouped_gemm_t_supported(const GemmLaunch& L);
 bool grouped_gemm_t_preferred(const GemmLaunch& L);
+cudaError_t launch_grouped_gemm_pair(const GemmLaunch& L, cudaStream_t stream);
+bool grouped_gemm_pair_supported(const GemmLaunch& L);
+bool grouped_gemm_pair_preferred(const GemmLaunch& L);
 
 cudaError_t launch_route_topk(const float* logits, int T, int E, int k, int score_fn,
                               int renormalize, int32_t* ids, float* weights, cudaStream_t stream);

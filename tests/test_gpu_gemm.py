@@ -64,10 +64,26 @@ GEMM_CASES = [
     (200, 8, 2, 256, 384, None),
     (260, 8, 3, 512, 128, [0, 1, 127, 128, 129, 0, 255, 140]),
     (300, 5, 1, 192, 256, [0, 0, 300, 0, 0]),
+    # more tiles than resident CTAs: every persistent loop wraps
+    (2048, 16, 4, 512, 512, None),
 ]
 
 
-TILINGS = [0x10, 0x20]   # MOE_TILE_TOKEN_ROWS, MOE_TILE_WEIGHT_ROWS
+# MOE_TILE_TOKEN_ROWS, MOE_TILE_WEIGHT_ROWS, MOE_TILE_WEIGHT_ROWS_PAIR
+TILINGS = [0x10, 0x20, 0x30]
+PAIR = 0x30
+
+
+def _pair_unsupported(tiling, N, fp8=False):
+    """The pair tiling takes bf16 operands with N % 256 == 0 only."""
+    return tiling == PAIR and (fp8 or N % 256 != 0)
+
+
+def _expect_unsupported(call):
+    import moe_routed_expert_top_b200 as M
+    with pytest.raises(M.MoeError) as ei:
+        call()
+    assert ei.value.status == M.MOE_ERR_UNSUPPORTED
 
 
 @pytest.mark.parametrize("tiling", TILINGS)
@@ -80,9 +96,13 @@ def test_grouped_gemm_store(T, E, k, H, F, sizes, f32, tiling):
     prob = gu.problem(cfg)
     C = torch.full((L["P"], 2 * F), float("nan"), dtype=torch.float32 if f32 else torch.bfloat16,
                    device="cuda")
-    M.moe_grouped_gemm(prob, 0, 2 * F, H, x_perm, None, wgu, None, tables,
-                       (M.MOE_EPI_STORE_F32 if f32 else M.MOE_EPI_STORE) | tiling, C, None, None,
-                       status)
+    call = lambda: M.moe_grouped_gemm(prob, 0, 2 * F, H, x_perm, None, wgu, None, tables,
+                                      (M.MOE_EPI_STORE_F32 if f32 else M.MOE_EPI_STORE) | tiling,
+                                      C, None, None, status)
+    if _pair_unsupported(tiling, 2 * F):
+        _expect_unsupported(call)
+        return
+    call()
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     refC = _oracle_rows_gemm(hidden, wgu, ref, E, k)
@@ -101,8 +121,12 @@ def test_grouped_gemm_swiglu(T, E, k, H, F, sizes, tiling):
     cfg, ids, hidden, L, tables, status, x_perm, ref, wgu, wd = _setup(T, E, k, H, F, 2, sizes)
     prob = gu.problem(cfg)
     h = torch.full((L["P"], F), float("nan"), dtype=torch.bfloat16, device="cuda")
-    M.moe_grouped_gemm(prob, 0, 2 * F, H, x_perm, None, wgu, None, tables,
-                       M.MOE_EPI_SWIGLU | tiling, h, None, None, status)
+    call = lambda: M.moe_grouped_gemm(prob, 0, 2 * F, H, x_perm, None, wgu, None, tables,
+                                      M.MOE_EPI_SWIGLU | tiling, h, None, None, status)
+    if _pair_unsupported(tiling, 2 * F):
+        _expect_unsupported(call)
+        return
+    call()
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     G = _oracle_rows_gemm(hidden, wgu, ref, E, k)
@@ -165,10 +189,15 @@ def test_grouped_gemm_fp8_block_scaled(T, E, k, H, F, sizes, tiling):
     for f32 in (False, True):
         y = torch.full((P, H), float("nan"), dtype=torch.float32 if f32 else torch.bfloat16,
                        device="cuda")
-        M.moe_grouped_gemm(prob, 0, H, F, torch.from_numpy(qa).cuda(), torch.from_numpy(sa).cuda(),
-                           torch.from_numpy(wq).cuda(), torch.from_numpy(ws).cuda(), tables,
-                           (M.MOE_EPI_STORE_F32 if f32 else M.MOE_EPI_STORE) | tiling, y, None,
-                           None, status)
+        call = lambda: M.moe_grouped_gemm(prob, 0, H, F, torch.from_numpy(qa).cuda(),
+                                          torch.from_numpy(sa).cuda(), torch.from_numpy(wq).cuda(),
+                                          torch.from_numpy(ws).cuda(), tables,
+                                          (M.MOE_EPI_STORE_F32 if f32 else M.MOE_EPI_STORE) | tiling,
+                                          y, None, None, status)
+        if _pair_unsupported(tiling, H, fp8=True):
+            _expect_unsupported(call)
+            continue
+        call()
         torch.cuda.synchronize()
         assert int(status.item()) == 0
         if f32:
@@ -188,8 +217,12 @@ def test_dense_gemm_store(M_rows, N, K, tiling):
     B = (torch.randn(N, K, generator=g, device="cuda") * 0.05).to(torch.bfloat16)
     C = torch.empty(M_rows, N, dtype=torch.bfloat16, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    M.moe_grouped_gemm(None, M_rows, N, K, A, None, B, None, None, M.MOE_EPI_STORE | tiling, C,
-                       None, None, status)
+    call = lambda: M.moe_grouped_gemm(None, M_rows, N, K, A, None, B, None, None,
+                                      M.MOE_EPI_STORE | tiling, C, None, None, status)
+    if _pair_unsupported(tiling, N):
+        _expect_unsupported(call)
+        return
+    call()
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     gu.assert_within_tol(gu.f64(C), gu.f64(A) @ gu.f64(B).T, "dense")
