@@ -121,6 +121,18 @@ enum {
   MOE_TILE_WEIGHT_ROWS_PAIR = 0x30
 };
 
+/* Flag OR-ed into moe_grouped_gemm's `epilogue`: the permutation is fused into
+ * the GEMM. A is then the hidden states bf16 [prob->T, K] (K == prob->H) and
+ * row r of the grouped problem is A[pair_of_row[r] / top_k] (pair_of_row from
+ * `tables`), the rows x_perm would hold (TileOPs PR #1580, copy elimination;
+ * TileLang tutorial "Example 07", section 1, permutation). Grouped mode, bf16,
+ * the weight-row pair tiling only (MOE_TILE_AUTO or MOE_TILE_WEIGHT_ROWS_PAIR
+ * with its shape rules), else MOE_ERR_UNSUPPORTED; without tables
+ * MOE_ERR_INVALID_ARG. The rows are fetched with four-row TMA gathers once per
+ * weight block; on B200 this measured slower than writing x_perm once with
+ * moe_route_permute, so moe_experts_forward does not use it. */
+enum { MOE_A_GATHER = 0x100 };
+
 /* One MoE layer's shape and routing options. */
 typedef struct moe_problem {
   int32_t T;            /* tokens (>= 0; 0 is a no-op) */

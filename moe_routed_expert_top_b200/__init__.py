@@ -34,6 +34,7 @@ MOE_SCORE_SOFTMAX, MOE_SCORE_SIGMOID = 0, 1
 MOE_EPI_STORE, MOE_EPI_SWIGLU, MOE_EPI_SWIGLU_FP8, MOE_EPI_STORE_F32 = 0, 1, 2, 3
 MOE_TILE_AUTO, MOE_TILE_TOKEN_ROWS, MOE_TILE_WEIGHT_ROWS = 0x00, 0x10, 0x20
 MOE_TILE_WEIGHT_ROWS_PAIR = 0x30
+MOE_A_GATHER = 0x100  # moe_grouped_gemm: A = hidden states, rows gathered through the tables
 
 EXPORTED_SYMBOLS = (
     "moe_get_tables_layout", "moe_workspace_bytes", "moe_route_topk", "moe_route_permute",

@@ -633,7 +633,8 @@ static cudaError_t run_gemm(const GemmLaunch& L, cudaStream_t stream) {
 }
 
 cudaError_t launch_grouped_gemm(const GemmLaunch& L, cudaStream_t stream) {
-  if (L.tiling == kTilingWeightsPair || (L.tiling == kTilingAuto && grouped_gemm_pair_preferred(L)))
+  if (L.gather || L.tiling == kTilingWeightsPair ||
+      (L.tiling == kTilingAuto && grouped_gemm_pair_preferred(L)))
     return grouped_gemm_pair_supported(L) ? launch_grouped_gemm_pair(L, stream)
                                           : cudaErrorNotSupported;
   if (grouped_gemm_t_supported(L) &&

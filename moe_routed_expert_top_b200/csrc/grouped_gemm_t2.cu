@@ -55,6 +55,11 @@ struct PParams {
   int ldc;
   int out_f32;
   int32_t* status;
+  // gather mode: token row r is hidden[pair_of_row[r] / top_k] (K columns)
+  const __nv_bfloat16* hidden;
+  const int32_t* pair_of_row;
+  int top_k;
+  int hidden_rows;
 };
 
 __host__ __device__ constexpr int pmin(int a, int b) { return a < b ? a : b; }
@@ -130,8 +135,11 @@ __device__ __forceinline__ void pair_commit(uint32_t bar) {
                : "memory");
 }
 
-template <int kMode, int TN>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+// Threads per CTA: producer warp, MMA warp, 4 epilogue warps.
+constexpr int kPairThreads = 192;
+
+template <int kMode, int TN, bool kGather>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmW,
                              const __grid_constant__ CUtensorMap tmX0,
                              const __grid_constant__ CUtensorMap tmX1,
@@ -140,6 +148,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   using Cfg = PCfg<kMode, TN>;
   constexpr int STAGES = Cfg::STAGES;
   constexpr int NUM_ACC = Cfg::NUM_ACC;
+  constexpr int kThreads = kPairThreads;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -191,7 +200,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   }
   if (warp == 1) tmem_alloc_pair(smem_u32(tmem_slot), Cfg::TMEM_COLS);
   {
-    const int per = (E + 191) / 192;
+    const int per = (E + kThreads - 1) / kThreads;
     const int beg = threadIdx.x * per;
     int local = 0;
     for (int i = 0; i < per && beg + i < E; ++i) {
@@ -215,7 +224,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       const int s = p.group_sizes ? __ldg(p.group_sizes + beg + i) : p.M_dense;
       run += (s + TN - 1) / TN;
     }
-    if (threadIdx.x == 191) cpre[E] = before + inc;
+    if (threadIdx.x == kThreads - 1) cpre[E] = before + inc;
   }
   tc_fence_before();
   __syncthreads();
@@ -229,7 +238,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
-    if (lane == 0) {
+    // Lane 0 waits for free stages and loads the weight rows (and the token
+    // rows as one box). Gather mode: the token rows are hidden-state rows
+    // picked through pair_of_row, and lane l fetches rows 4l..4l+3 of this
+    // CTA's half with one four-row TMA gather (512 B of the 128-byte-swizzled
+    // tile: the same bytes in the same place as the box load).
+    if (kGather || lane == 0) {
       const uint64_t pol_act = l2_policy_evict_last();
       const uint64_t pol_w1 = l2_policy_by_code(MOE_W_POLICY_SINGLE);
       const uint64_t pol_wn = l2_policy_by_code(MOE_W_POLICY_MULTI);
@@ -243,28 +257,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         const int nmma = (ti.nt + 31) & ~31;
         const int half = nmma / 2;
         const int xb = half_box(half);
-        const uint32_t bytes_pair = 2u * (Cfg::A_BYTES + (16u << xb) * 128u);
+        const uint32_t x_bytes = kGather ? static_cast<uint32_t>(half) * 128u : (16u << xb) * 128u;
+        const uint32_t bytes_pair = 2u * (Cfg::A_BYTES + x_bytes);
         const int wrow = ti.e * p.N + ti.wb * Cfg::PAIR_COLS +
                          static_cast<int>(rank) * (kMode == kPSwiglu ? 64 : 128);
         const uint64_t pol_w = ti.chunks > 1 ? pol_wn : pol_w1;
         const int trow = ti.m0 + static_cast<int>(rank) * half;
+        const bool gather_lane = kGather && 4 * lane < half;
+        int g[4] = {0, 0, 0, 0};
+        if (gather_lane) {
+          // rows past the tile's tokens repeat its first token: they only feed
+          // MMA columns that are never stored
+          auto token_of = [&](int row) {
+            const int v = __ldg(p.pair_of_row + row) / p.top_k;
+            return v < 0 ? 0 : (v >= p.hidden_rows ? p.hidden_rows - 1 : v);
+          };
+          const int first = token_of(ti.m0);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int i = trow - ti.m0 + 4 * lane + j;  // row within the tile
+            g[j] = i < ti.nt ? token_of(ti.m0 + i) : first;
+          }
+        }
         for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.status)) {
+          uint32_t got = 1;
+          if (lane == 0) got = mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.status);
+          if constexpr (kGather) got = __shfl_sync(0xffffffffu, got, 0);
+          if (!got) {
             ok = false;
             break;
           }
           const uint32_t fb_local = full0 + 8 * stage;
           const uint32_t fb = cluster_map_shared(fb_local, 0);
-          if (leader) mbar_arrive_expect_tx(fb_local, bytes_pair);
-          const uint32_t a_dst = smem_u32(sA + stage * Cfg::A_BYTES);
-          if constexpr (kMode == kPSwiglu) {
-            tma_load_2d_pair(a_dst, &tmW, kb * Cfg::BK, wrow, fb, pol_w);
-            tma_load_2d_pair(a_dst + 64 * 128, &tmW, kb * Cfg::BK, wrow + p.N / 2, fb, pol_w);
-          } else {
-            tma_load_2d_pair(a_dst, &tmW, kb * Cfg::BK, wrow, fb, pol_w);
+          const uint32_t b_dst = smem_u32(sB + stage * Cfg::B_BYTES);
+          if (lane == 0) {
+            if (leader) mbar_arrive_expect_tx(fb_local, bytes_pair);
+            const uint32_t a_dst = smem_u32(sA + stage * Cfg::A_BYTES);
+            if constexpr (kMode == kPSwiglu) {
+              tma_load_2d_pair(a_dst, &tmW, kb * Cfg::BK, wrow, fb, pol_w);
+              tma_load_2d_pair(a_dst + 64 * 128, &tmW, kb * Cfg::BK, wrow + p.N / 2, fb, pol_w);
+            } else {
+              tma_load_2d_pair(a_dst, &tmW, kb * Cfg::BK, wrow, fb, pol_w);
+            }
+            if constexpr (!kGather)
+              tma_load_2d_pair(b_dst, xmaps[xb], kb * Cfg::BK, trow, fb, pol_act);
           }
-          tma_load_2d_pair(smem_u32(sB + stage * Cfg::B_BYTES), xmaps[xb], kb * Cfg::BK, trow, fb,
-                           pol_act);
+          if (gather_lane)
+            tma_gather4_pair(b_dst + lane * 512, &tmX0, kb * Cfg::BK, g[0], g[1], g[2], g[3], fb,
+                             pol_act);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -272,7 +312,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         }
       }
       // every load this CTA issued has been consumed (its stage released) before leaving
-      if (ok) {
+      if (ok && lane == 0) {
         for (int i = 0; i < STAGES; ++i) {
           mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.status);
           if (++stage == STAGES) {
@@ -455,35 +495,40 @@ bool p_encode(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows, uin
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int kMode, int TN>
+template <int kMode, int TN, bool kGather>
 cudaError_t run_pair(const GemmLaunch& L, cudaStream_t stream) {
   using Cfg = PCfg<kMode, TN>;
+  constexpr int kThreads = kPairThreads;
   static int max_pairs_cache[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (max_pairs_cache[dev] == 0) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_pair_kernel<kMode, TN>,
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_pair_kernel<kMode, TN, kGather>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Cfg::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     // pairs that can be resident at once (a pair needs both SMs of one TPC free)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(device_sm_count() & ~1));
-    cfg.blockDim = dim3(192);
+    cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
     int n = 0;
-    e = cudaOccupancyMaxActiveClusters(&n, grouped_gemm_pair_kernel<kMode, TN>, &cfg);
+    e = cudaOccupancyMaxActiveClusters(&n, grouped_gemm_pair_kernel<kMode, TN, kGather>, &cfg);
     if (e != cudaSuccess) return e;
     max_pairs_cache[dev] = n > 0 ? n : 1;
   }
   const bool grouped = L.group_sizes != nullptr;
   const int E = grouped ? L.E : 1;
+  // rows of the A operand in memory: the hidden states in gather mode
+  const int a_rows = kGather ? L.a_rows : L.rows;
   CUtensorMap tmW, tmX[kPXBoxes];
   if (!p_encode(&tmW, L.B, L.K, static_cast<uint64_t>(E) * L.N, kMode == kPSwiglu ? 64 : 128))
     return cudaErrorInvalidValue;
+  // gather mode: map 0 is the hidden states with a one-row-high box (four-row gathers)
   for (int i = 0; i < kPXBoxes; ++i)
-    if (!p_encode(&tmX[i], L.A, L.K, L.rows, 16u << i)) return cudaErrorInvalidValue;
+    if (!p_encode(&tmX[i], L.A, L.K, a_rows, kGather && i == 0 ? 1u : 16u << i))
+      return cudaErrorInvalidValue;
   PParams p{};
   p.M_dense = grouped ? 0 : L.rows;
   p.N = L.N;
@@ -496,21 +541,34 @@ cudaError_t run_pair(const GemmLaunch& L, cudaStream_t stream) {
   p.ldc = kMode == kPSwiglu ? L.N / 2 : L.N;
   p.out_f32 = L.out_f32;
   p.status = L.status;
+  p.hidden = static_cast<const __nv_bfloat16*>(L.A);
+  p.pair_of_row = L.pair_of_row;
+  p.top_k = L.top_k;
+  p.hidden_rows = a_rows;
   const int WB = kMode == kPSwiglu ? (L.N / 2) / 128 : L.N / 256;
   const long long chunks_ub = grouped ? (static_cast<long long>(L.rows) + TN - 1) / TN + E
                                       : (static_cast<long long>(L.rows) + TN - 1) / TN;
   const long long pairs_ub = chunks_ub * WB;
   const int max_pairs = max_pairs_cache[dev];
   const int pairs = static_cast<int>(pairs_ub < max_pairs ? (pairs_ub > 0 ? pairs_ub : 1) : max_pairs);
-  grouped_gemm_pair_kernel<kMode, TN><<<2 * pairs, 192, Cfg::SMEM_BYTES, stream>>>(
+  grouped_gemm_pair_kernel<kMode, TN, kGather><<<2 * pairs, kThreads, Cfg::SMEM_BYTES, stream>>>(
       tmW, tmX[0], tmX[1], tmX[2], tmX[3], p);
   return cudaGetLastError();
+}
+
+template <int kMode, int TN>
+cudaError_t run_pair_g(const GemmLaunch& L, cudaStream_t stream) {
+  return L.gather ? run_pair<kMode, TN, true>(L, stream) : run_pair<kMode, TN, false>(L, stream);
 }
 
 }  // namespace
 
 bool grouped_gemm_pair_supported(const GemmLaunch& L) {
   if (L.A_scales != nullptr || L.B_scales != nullptr || L.E > 1024) return false;
+  // gathering needs the group tables and the row -> pair map
+  if (L.gather && (L.group_sizes == nullptr || L.pair_of_row == nullptr || L.top_k <= 0 ||
+                   L.a_rows <= 0))
+    return false;
   if (L.mode == kModeStore) return L.N % 256 == 0 && L.K % 64 == 0;
   if (L.mode == kModeSwiglu) return (L.N / 2) % 128 == 0 && L.K % 64 == 0;
   return false;
@@ -529,9 +587,9 @@ bool grouped_gemm_pair_preferred(const GemmLaunch& L) {
 cudaError_t launch_grouped_gemm_pair(const GemmLaunch& L, cudaStream_t stream) {
   const bool small = L.group_sizes != nullptr && L.rows <= 64 * L.E;
   if (L.mode == kModeSwiglu)
-    return small ? run_pair<kPSwiglu, 64>(L, stream) : run_pair<kPSwiglu, 256>(L, stream);
+    return small ? run_pair_g<kPSwiglu, 64>(L, stream) : run_pair_g<kPSwiglu, 256>(L, stream);
   if (L.mode == kModeStore)
-    return small ? run_pair<kPStore, 64>(L, stream) : run_pair<kPStore, 256>(L, stream);
+    return small ? run_pair_g<kPStore, 64>(L, stream) : run_pair_g<kPStore, 256>(L, stream);
   return cudaErrorInvalidValue;
 }
 

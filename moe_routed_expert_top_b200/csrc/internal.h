@@ -32,6 +32,12 @@ struct GemmLaunch {
   float* C_scales = nullptr;
   float* debug_h = nullptr;
   int32_t* status = nullptr;
+  // gather mode (weight-row pair tiling only): A is the hidden states
+  // [a_rows, K] and row r of the grouped problem is A[pair_of_row[r] / top_k]
+  int gather = 0;
+  const int32_t* pair_of_row = nullptr;
+  int top_k = 0;
+  int a_rows = 0;
 };
 
 // Tiling of the grouped GEMM: token-row tiles (grouped_gemm.cu), weight-row

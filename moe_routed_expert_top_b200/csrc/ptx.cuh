@@ -148,11 +148,26 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t smem_dst, const void* 
       : "memory");
 }
 
+// Gather four rows (y0..y3, one-row-high box of the tensor map) at inner
+// coordinate x into 4 consecutive 128-byte rows of this CTA's shared memory
+// (swizzled by address like any box), completing on a barrier that may live in
+// the pair's leader CTA.
+__device__ __forceinline__ void tma_gather4_pair(uint32_t smem_dst, const void* tmap, int32_t x,
+                                                 int32_t y0, int32_t y1, int32_t y2, int32_t y3,
+                                                 uint32_t bar_cluster, uint64_t cache_hint) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::"
+      "complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(
+          smem_dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3),
+      "r"(bar_cluster), "l"(cache_hint)
+      : "memory");
+}
+
 // Arrive on an mbarrier addressed in the cluster shared window (possibly the peer's).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
 }
-
 // L2 eviction-priority hints (createpolicy fractions of 1.0).
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t p;

@@ -133,6 +133,63 @@ def test_grouped_gemm_swiglu(T, E, k, H, F, sizes, tiling):
     gu.assert_within_tol(gu.f64(h), O.bf16_round(O.swiglu(G, F)), "swiglu epilogue")
 
 
+@pytest.mark.parametrize("epi", ["store_f32", "swiglu"])
+@pytest.mark.parametrize("T,E,k,H,F,sizes", [c for c in GEMM_CASES if c[4] % 128 == 0])
+def test_grouped_gemm_gather(T, E, k, H, F, sizes, epi):
+    """The permutation fused into the gate+up GEMM (MOE_A_GATHER): A is the
+    hidden states and row r is hidden[pair_of_row[r] / k]. Against the oracle
+    (which permutes on its own), and bit-identical to the same tiling fed the
+    explicitly permuted rows."""
+    gu = _gu()
+    import moe_routed_expert_top_b200 as M
+    cfg, ids, hidden, L, tables, status, x_perm, ref, wgu, wd = _setup(T, E, k, H, F, 5, sizes)
+    prob = gu.problem(cfg)
+    P = L["P"]
+    f32 = epi == "store_f32"
+    flag = M.MOE_EPI_STORE_F32 if f32 else M.MOE_EPI_SWIGLU
+    shape = (P, 2 * F) if f32 else (P, F)
+    dt = torch.float32 if f32 else torch.bfloat16
+    out_g = torch.full(shape, float("nan"), dtype=dt, device="cuda")
+    out_x = torch.full(shape, float("nan"), dtype=dt, device="cuda")
+    for tiling in (M.MOE_TILE_AUTO, PAIR):
+        M.moe_grouped_gemm(prob, 0, 2 * F, H, hidden, None, wgu, None, tables,
+                           flag | tiling | M.MOE_A_GATHER, out_g, None, None, status)
+        M.moe_grouped_gemm(prob, 0, 2 * F, H, x_perm, None, wgu, None, tables, flag | PAIR,
+                           out_x, None, None, status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        assert torch.equal(out_g.view(torch.int32 if f32 else torch.int16),
+                           out_x.view(torch.int32 if f32 else torch.int16))
+    G = _oracle_rows_gemm(hidden, wgu, ref, E, k)
+    if f32:
+        gu.assert_within_tol(gu.f64(out_g), G, "gathered gate_up f32", rtol=1e-4, atol=1e-4)
+    else:
+        gu.assert_within_tol(gu.f64(out_g), O.bf16_round(O.swiglu(G, F)), "gathered swiglu")
+
+
+def test_grouped_gemm_gather_rejects():
+    gu = _gu()
+    import moe_routed_expert_top_b200 as M
+    T, E, k, H, F = 200, 8, 2, 256, 384
+    cfg, ids, hidden, L, tables, status, x_perm, ref, wgu, wd = _setup(T, E, k, H, F, 6)
+    prob = gu.problem(cfg)
+    h = torch.empty(L["P"], F, dtype=torch.bfloat16, device="cuda")
+    # another tiling
+    _expect_unsupported(lambda: M.moe_grouped_gemm(
+        prob, 0, 2 * F, H, hidden, None, wgu, None, tables,
+        M.MOE_EPI_SWIGLU | M.MOE_TILE_WEIGHT_ROWS | M.MOE_A_GATHER, h, None, None, status))
+    # no tables to gather through; K other than H
+    for call in (lambda: M.moe_grouped_gemm(None, T, 2 * F, H, hidden, None, wgu, None, None,
+                                            M.MOE_EPI_SWIGLU | M.MOE_A_GATHER, h, None, None,
+                                            status),
+                 lambda: M.moe_grouped_gemm(prob, 0, 2 * F, H - 64, hidden, None, wgu, None,
+                                            tables, M.MOE_EPI_SWIGLU | M.MOE_A_GATHER, h, None,
+                                            None, status)):
+        with pytest.raises(M.MoeError) as ei:
+            call()
+        assert ei.value.status == M.MOE_ERR_INVALID_ARG
+
+
 @pytest.mark.parametrize("T,E,k,H,F,sizes", [c for c in GEMM_CASES if c[4] % 128 == 0])
 def test_grouped_gemm_swiglu_fp8_epilogue(T, E, k, H, F, sizes):
     gu = _gu()
