@@ -285,6 +285,30 @@ moe_status moe_experts_forward(const moe_problem* prob, const void* hidden,
                                float scale, void* out, void* workspace, size_t ws_bytes,
                                moe_stream_t stream);
 
+/* One tensor-parallel rank's share of the shared expert, a dense SwiGLU MLP on
+ * all tokens (TileOPs PR #778 "SharedFusedMoE with native shared expert kernel
+ * and TP support": Design, TP split convention, Partial output contract).
+ * The caller passes the COMPLETE weights; rank r of tp_size owns
+ * F_p = F_s / tp_size FFN columns:
+ *   gate rows [r*F_p, (r+1)*F_p) and up rows F_s + [r*F_p, (r+1)*F_p) of
+ *   w_gate_up bf16 [2*F_s, H] (column parallel), and columns
+ *   [r*F_p, (r+1)*F_p) of w_down bf16 [H, F_s] (row parallel),
+ * all read in place (no slice copies), and writes
+ *   out [T, H] = bf16(SiLU(x Wg^T) * (x Wu^T)) Wd^T   (this rank's slices)
+ * as fp32 (out_f32 = 1) or bf16 (0). With tp_size > 1, `out` is a partial
+ * sum: the caller all-reduces it over the ranks and adds the routed output.
+ * Errors: null or unaligned pointers, T < 0, H or F_p not a multiple of 64,
+ * tp_rank outside [0, tp_size), F_s % tp_size != 0 -> MOE_ERR_INVALID_ARG;
+ * tp_size > 1 also needs H % 256 == 0 and F_p % 128 == 0, else
+ * MOE_ERR_UNSUPPORTED; ws_bytes < moe_shared_workspace_bytes ->
+ * MOE_ERR_WORKSPACE. `workspace` holds h and the device status word (its
+ * first int32, zeroed by the call). T == 0 enqueues nothing. */
+size_t moe_shared_workspace_bytes(int32_t T, int32_t H, int32_t F_s, int32_t tp_size);
+moe_status moe_shared_expert_forward(int32_t T, int32_t H, int32_t F_s, int32_t tp_size,
+                                     int32_t tp_rank, const void* hidden, const void* w_gate_up,
+                                     const void* w_down, int32_t out_f32, void* out,
+                                     void* workspace, size_t ws_bytes, moe_stream_t stream);
+
 /* Capacity of the library's built-in scratch area used by
  * moe_experts_forward_noalloc: 64 MiB of device memory. */
 #define MOE_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)

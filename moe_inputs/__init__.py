@@ -75,6 +75,14 @@ CONFIGS = {
     "dsv3_decode_fp8": MoeConfig("dsv3_decode_fp8", T=512, E=256, top_k=8, H=7168, F=2048,
                                  score_fn="sigmoid", logits="zipf",
                                  routed_scaling_factor=2.5, down_fp8=True, seed=4),
+    # Kimi-K2-scale layer with its large shared expert (TileOPs PR #778
+    # "SharedFusedMoE with native shared expert kernel and TP support",
+    # Benchmark: E=384, top-8, H=7168, F=2048, F_s=18432, sigmoid, tokens
+    # 1..4096); routed_scaling_factor 2.827 as in the end-to-end linearity check
+    # of TileOPs PR #1580 (Test Plan)
+    "kimi_k2": MoeConfig("kimi_k2", T=512, E=384, top_k=8, H=7168, F=2048,
+                         score_fn="sigmoid", logits="normal", routed_scaling_factor=2.827,
+                         F_shared=18432, seed=5),
 }
 
 

@@ -18,7 +18,8 @@ __all__ = [
     "moe_get_tables_layout", "moe_workspace_bytes", "moe_route_topk", "moe_route_permute",
     "moe_grouped_gemm", "moe_swiglu_quant", "moe_unpermute", "moe_quantize_weight_128x128",
     "moe_experts_forward", "moe_decode_device_status", "moe_status_string",
-    "moe_last_launch_count", "EXPORTED_SYMBOLS",
+    "moe_last_launch_count", "moe_shared_workspace_bytes", "moe_shared_expert_forward",
+    "EXPORTED_SYMBOLS",
     "MOE_OK", "MOE_EPI_STORE", "MOE_EPI_SWIGLU", "MOE_EPI_SWIGLU_FP8", "MOE_EPI_STORE_F32",
     "MOE_SCORE_SOFTMAX", "MOE_SCORE_SIGMOID", "MOE_DEV_BAD_EXPERT_ID", "MOE_DEV_TIMEOUT",
 ]
@@ -41,6 +42,7 @@ EXPORTED_SYMBOLS = (
     "moe_grouped_gemm", "moe_swiglu_quant", "moe_unpermute", "moe_quantize_weight_128x128",
     "moe_experts_forward", "moe_decode_device_status", "moe_status_string",
     "moe_last_cuda_error", "moe_last_launch_count", "moe_experts_forward_noalloc",
+    "moe_shared_workspace_bytes", "moe_shared_expert_forward",
 )
 
 
@@ -114,6 +116,11 @@ def lib() -> ctypes.CDLL:
                                                ctypes.c_float, _P, _P, ctypes.c_size_t, _P]),
         "moe_experts_forward_noalloc": (ctypes.c_int, [PP, _P, _P, _P, _P, _P, _P, _P, _P,
                                                        ctypes.c_float, _P, _P]),
+        "moe_shared_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int32] * 4),
+        "moe_shared_expert_forward": (ctypes.c_int, [ctypes.c_int32] * 5 + [_P, _P, _P,
+                                                                            ctypes.c_int32, _P,
+                                                                            _P, ctypes.c_size_t,
+                                                                            _P]),
         "moe_decode_device_status": (ctypes.c_int, [ctypes.c_int32]),
         "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "moe_last_cuda_error": (ctypes.c_char_p, []),
@@ -217,6 +224,21 @@ def moe_experts_forward(prob, hidden, topk_ids, topk_weights, w_gate_up, w_down,
                                      _ptr(w_down_scales), _ptr(ws_gate_up), _ptr(ws_down),
                                      float(scale), _ptr(out), _ptr(workspace), int(ws_bytes),
                                      _stream(stream)), "moe_experts_forward")
+
+
+def moe_shared_workspace_bytes(T, H, F_s, tp_size=1) -> int:
+    return int(lib().moe_shared_workspace_bytes(int(T), int(H), int(F_s), int(tp_size)))
+
+
+def moe_shared_expert_forward(T, H, F_s, tp_size, tp_rank, hidden, w_gate_up, w_down, out_f32,
+                              out, workspace, ws_bytes=None, stream=None):
+    if ws_bytes is None:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().moe_shared_expert_forward(int(T), int(H), int(F_s), int(tp_size), int(tp_rank),
+                                           _ptr(hidden), _ptr(w_gate_up), _ptr(w_down),
+                                           int(out_f32), _ptr(out), _ptr(workspace),
+                                           int(ws_bytes), _stream(stream)),
+           "moe_shared_expert_forward")
 
 
 def moe_decode_device_status(dev_status: int) -> int:

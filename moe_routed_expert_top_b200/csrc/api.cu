@@ -414,6 +414,72 @@ moe_status moe_experts_forward(const moe_problem* prob, const void* hidden,
   return MOE_OK;
 }
 
+size_t moe_shared_workspace_bytes(int32_t T, int32_t H, int32_t F_s, int32_t tp_size) {
+  if (T < 0 || H <= 0 || F_s <= 0 || tp_size <= 0 || F_s % tp_size != 0) return 0;
+  const int64_t Fp = F_s / tp_size;
+  return static_cast<size_t>(1024 + round_up(static_cast<int64_t>(T) * Fp * 2, 1024));
+}
+
+moe_status moe_shared_expert_forward(int32_t T, int32_t H, int32_t F_s, int32_t tp_size,
+                                     int32_t tp_rank, const void* hidden, const void* w_gate_up,
+                                     const void* w_down, int32_t out_f32, void* out,
+                                     void* workspace, size_t ws_bytes, moe_stream_t stream) {
+  if (hidden == nullptr || w_gate_up == nullptr || w_down == nullptr || out == nullptr ||
+      workspace == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(hidden) || !aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(out) ||
+      !aligned16(workspace))
+    return MOE_ERR_INVALID_ARG;
+  if (T < 0 || H <= 0 || H % 64 != 0 || F_s <= 0 || tp_size <= 0 || tp_rank < 0 ||
+      tp_rank >= tp_size || F_s % tp_size != 0)
+    return MOE_ERR_INVALID_ARG;
+  const int64_t Fp = F_s / tp_size;
+  if (Fp % 64 != 0) return MOE_ERR_INVALID_ARG;
+  if (tp_size > 1 && (H % 256 != 0 || Fp % 128 != 0)) return MOE_ERR_UNSUPPORTED;
+  if (ws_bytes < moe_shared_workspace_bytes(T, H, F_s, tp_size)) return MOE_ERR_WORKSPACE;
+  g_last_launches = 0;
+  if (T == 0) return MOE_OK;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  int32_t* status = reinterpret_cast<int32_t*>(base);
+  void* h = base + 1024;
+  MOE_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int32_t), st));
+  const size_t r = static_cast<size_t>(tp_rank);
+  // gate+up with the SwiGLU epilogue: this rank's gate rows and, F_s rows
+  // further, its up rows, addressed in the complete w_gate_up
+  moe::GemmLaunch d;
+  d.rows = T;
+  d.E = 1;
+  d.status = status;
+  d.mode = moe::kModeSwiglu;
+  d.N = static_cast<int>(2 * Fp);
+  d.K = H;
+  d.A = hidden;
+  d.B = static_cast<const uint16_t*>(w_gate_up) + r * Fp * H;  // bf16 elements
+  if (tp_size > 1) {
+    d.up_off = F_s;
+    d.b_rows = 2LL * F_s - static_cast<long long>(r) * Fp;
+  }
+  d.C = h;
+  if (tp_size > 1 && !moe::grouped_gemm_pair_supported(d)) return MOE_ERR_UNSUPPORTED;
+  MOE_CUDA_TRY(moe::launch_grouped_gemm(d, st));
+  // down: this rank's F_p columns of the complete w_down (row pitch F_s)
+  d.mode = moe::kModeStore;
+  d.N = H;
+  d.K = static_cast<int>(Fp);
+  d.A = h;
+  d.B = static_cast<const uint16_t*>(w_down) + r * Fp;
+  d.up_off = 0;
+  d.b_rows = 0;
+  if (tp_size > 1) d.ldb = F_s;
+  d.C = out;
+  d.out_f32 = out_f32 != 0;
+  if (tp_size > 1 && !moe::grouped_gemm_pair_supported(d)) return MOE_ERR_UNSUPPORTED;
+  MOE_CUDA_TRY(moe::launch_grouped_gemm(d, st));
+  g_last_launches = 2;
+  return MOE_OK;
+}
+
 moe_status moe_decode_device_status(int32_t dev_status) {
   if (dev_status == 0) return MOE_OK;
   if (dev_status & MOE_DEV_TIMEOUT) return MOE_ERR_TIMEOUT;

@@ -633,7 +633,9 @@ static cudaError_t run_gemm(const GemmLaunch& L, cudaStream_t stream) {
 }
 
 cudaError_t launch_grouped_gemm(const GemmLaunch& L, cudaStream_t stream) {
-  if (L.gather || L.tiling == kTilingWeightsPair ||
+  // B as a strided view (a tensor-parallel shard) is read by the pair tiling only
+  const bool b_view = L.ldb != 0 || L.up_off != 0 || L.b_rows != 0;
+  if (L.gather || b_view || L.tiling == kTilingWeightsPair ||
       (L.tiling == kTilingAuto && grouped_gemm_pair_preferred(L)))
     return grouped_gemm_pair_supported(L) ? launch_grouped_gemm_pair(L, stream)
                                           : cudaErrorNotSupported;

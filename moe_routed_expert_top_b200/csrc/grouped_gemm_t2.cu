@@ -60,6 +60,7 @@ struct PParams {
   const int32_t* pair_of_row;
   int top_k;
   int hidden_rows;
+  int up_off;  // SwiGLU: rows from a gate row of W to its up row
 };
 
 __host__ __device__ constexpr int pmin(int a, int b) { return a < b ? a : b; }
@@ -295,7 +296,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             const uint32_t a_dst = smem_u32(sA + stage * Cfg::A_BYTES);
             if constexpr (kMode == kPSwiglu) {
               tma_load_2d_pair(a_dst, &tmW, kb * Cfg::BK, wrow, fb, pol_w);
-              tma_load_2d_pair(a_dst + 64 * 128, &tmW, kb * Cfg::BK, wrow + p.N / 2, fb, pol_w);
+              tma_load_2d_pair(a_dst + 64 * 128, &tmW, kb * Cfg::BK, wrow + p.up_off, fb, pol_w);
             } else {
               tma_load_2d_pair(a_dst, &tmW, kb * Cfg::BK, wrow, fb, pol_w);
             }
@@ -483,11 +484,13 @@ PFN_cuTensorMapEncodeTiled_v12000 p_encode_fn() {
   return fn;
 }
 
-bool p_encode(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows, uint32_t box_rows) {
+// Tensor map of a bf16 matrix of `rows` rows of K elements, `ld` elements apart.
+bool p_encode(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows, uint32_t box_rows,
+              uint64_t ld) {
   auto fn = p_encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {K, rows};
-  cuuint64_t strides[1] = {K * 2};
+  cuuint64_t strides[1] = {ld * 2};
   cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
@@ -523,11 +526,13 @@ cudaError_t run_pair(const GemmLaunch& L, cudaStream_t stream) {
   // rows of the A operand in memory: the hidden states in gather mode
   const int a_rows = kGather ? L.a_rows : L.rows;
   CUtensorMap tmW, tmX[kPXBoxes];
-  if (!p_encode(&tmW, L.B, L.K, static_cast<uint64_t>(E) * L.N, kMode == kPSwiglu ? 64 : 128))
+  const uint64_t b_rows = L.b_rows > 0 ? static_cast<uint64_t>(L.b_rows) : static_cast<uint64_t>(E) * L.N;
+  const uint64_t ldb = L.ldb > 0 ? static_cast<uint64_t>(L.ldb) : static_cast<uint64_t>(L.K);
+  if (!p_encode(&tmW, L.B, L.K, b_rows, kMode == kPSwiglu ? 64 : 128, ldb))
     return cudaErrorInvalidValue;
   // gather mode: map 0 is the hidden states with a one-row-high box (four-row gathers)
   for (int i = 0; i < kPXBoxes; ++i)
-    if (!p_encode(&tmX[i], L.A, L.K, a_rows, kGather && i == 0 ? 1u : 16u << i))
+    if (!p_encode(&tmX[i], L.A, L.K, a_rows, kGather && i == 0 ? 1u : 16u << i, L.K))
       return cudaErrorInvalidValue;
   PParams p{};
   p.M_dense = grouped ? 0 : L.rows;
@@ -545,6 +550,7 @@ cudaError_t run_pair(const GemmLaunch& L, cudaStream_t stream) {
   p.pair_of_row = L.pair_of_row;
   p.top_k = L.top_k;
   p.hidden_rows = a_rows;
+  p.up_off = L.up_off > 0 ? L.up_off : L.N / 2;
   const int WB = kMode == kPSwiglu ? (L.N / 2) / 128 : L.N / 256;
   const long long chunks_ub = grouped ? (static_cast<long long>(L.rows) + TN - 1) / TN + E
                                       : (static_cast<long long>(L.rows) + TN - 1) / TN;
@@ -569,7 +575,9 @@ bool grouped_gemm_pair_supported(const GemmLaunch& L) {
   if (L.gather && (L.group_sizes == nullptr || L.pair_of_row == nullptr || L.top_k <= 0 ||
                    L.a_rows <= 0))
     return false;
-  if (L.mode == kModeStore) return L.N % 256 == 0 && L.K % 64 == 0;
+  // a strided view of B: rows at least K long, 16-byte row pitch
+  if (L.ldb != 0 && (L.ldb < L.K || L.ldb % 8 != 0)) return false;
+  if (L.mode == kModeStore) return L.N % 256 == 0 && L.K % 64 == 0 && L.up_off == 0;
   if (L.mode == kModeSwiglu) return (L.N / 2) % 128 == 0 && L.K % 64 == 0;
   return false;
 }

@@ -38,6 +38,14 @@ struct GemmLaunch {
   const int32_t* pair_of_row = nullptr;
   int top_k = 0;
   int a_rows = 0;
+  // B as a view into a larger matrix (weight-row pair tiling only; 0 = the
+  // default): ldb = elements between consecutive B rows (default K); up_off =
+  // rows from a gate row to its up row in SwiGLU mode (default N / 2); b_rows =
+  // rows addressable from B (default E * N). A tensor-parallel shard of a
+  // complete weight is addressed in place this way.
+  int ldb = 0;
+  int up_off = 0;
+  long long b_rows = 0;
 };
 
 // Tiling of the grouped GEMM: token-row tiles (grouped_gemm.cu), weight-row

@@ -1,16 +1,20 @@
-"""A routed-experts layer object around ``moe_experts_forward``.
+"""Layer objects around the C entry points: ``RoutedExperts``
+(``moe_experts_forward``), ``SharedExpert`` (``moe_shared_expert_forward``,
+one tensor-parallel rank) and ``SharedFusedMoE`` (both, with the partial
+output contract).
 
-It owns the weights (device tensors), the problem description and a
-workspace buffer sized by ``moe_workspace_bytes``; ``forward`` only marshals
-pointers into the C entry point. FP8 down weights are prepared once with
-``moe_quantize_weight_128x128`` when ``down_fp8`` is set.
+Each owns its weights (device tensors) and a workspace buffer sized by the
+library; ``forward`` only marshals pointers into the C entry points. FP8 down
+weights are prepared once with ``moe_quantize_weight_128x128`` when
+``down_fp8`` is set.
 """
 from __future__ import annotations
 
 import torch
 
 from . import (make_problem, moe_experts_forward, moe_quantize_weight_128x128,
-               moe_route_topk, moe_workspace_bytes)
+               moe_route_topk, moe_shared_expert_forward, moe_shared_workspace_bytes,
+               moe_workspace_bytes)
 
 
 class RoutedExperts:
@@ -75,3 +79,75 @@ class RoutedExperts:
     def device_status(self) -> int:
         """The device status word of the last forward (synchronises)."""
         return int(self._ws[:4].view(torch.int32).item())
+
+
+class SharedExpert:
+    """One tensor-parallel rank's share of the shared expert (TileOPs PR #778
+    "SharedFusedMoE with native shared expert kernel and TP support": TP split
+    convention, Partial output contract). It takes the COMPLETE weights
+    w_gate_up [2*F_s, H] (gate rows, then up rows) and w_down [H, F_s]; the
+    library reads rank r's F_s / tp_size columns in place (column-parallel
+    gate/up rows, row-parallel down columns), with no slice copies.
+    ``forward`` returns this rank's partial output [T, H]: with tp_size > 1
+    the caller all-reduces it over the ranks (``SharedFusedMoE.combine``)."""
+
+    def __init__(self, w_gate_up: torch.Tensor, w_down: torch.Tensor, tp_size: int = 1,
+                 tp_rank: int = 0):
+        two_fs, H = w_gate_up.shape
+        self.F_s, self.H = two_fs // 2, H
+        if w_down.shape != (H, self.F_s):
+            raise ValueError("w_down must be [H, F_s]")
+        if tp_size < 1 or not 0 <= tp_rank < tp_size or self.F_s % tp_size:
+            raise ValueError("need 0 <= tp_rank < tp_size and F_s % tp_size == 0")
+        self.tp_size, self.tp_rank = tp_size, tp_rank
+        self.w_gate_up = w_gate_up.contiguous()
+        self.w_down = w_down.contiguous()
+        self._ws = None
+
+    def forward(self, hidden: torch.Tensor, out: torch.Tensor | None = None,
+                out_f32: bool = True) -> torch.Tensor:
+        T = hidden.shape[0]
+        if out is None:
+            out = torch.empty(T, self.H, dtype=torch.float32 if out_f32 else torch.bfloat16,
+                              device=hidden.device)
+        need = moe_shared_workspace_bytes(T, self.H, self.F_s, self.tp_size)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(max(need, 1024), dtype=torch.uint8, device=hidden.device)
+        moe_shared_expert_forward(T, self.H, self.F_s, self.tp_size, self.tp_rank, hidden,
+                                  self.w_gate_up, self.w_down, out.dtype == torch.float32, out,
+                                  self._ws)
+        return out
+
+    def device_status(self) -> int:
+        return int(self._ws[:4].view(torch.int32).item())
+
+
+class SharedFusedMoE:
+    """Routed experts plus a tensor-parallel shared expert, with the pages'
+    partial output contract (TileOPs PR #778): ``forward`` returns
+    ``(shared_partial, routed_out)``; the routed path is not sharded. With
+    tp_size > 1 the caller all-reduces ``shared_partial`` and adds
+    ``routed_out`` (``combine`` does both)."""
+
+    def __init__(self, routed: RoutedExperts, shared: SharedExpert | None):
+        if routed.F_shared:
+            raise ValueError("the routed layer must not carry the shared expert as well")
+        self.routed, self.shared = routed, shared
+
+    def forward(self, hidden: torch.Tensor, topk_ids: torch.Tensor, topk_weights: torch.Tensor):
+        routed_out = self.routed.forward(hidden, topk_ids, topk_weights)
+        shared_partial = None if self.shared is None else self.shared.forward(hidden)
+        return shared_partial, routed_out
+
+    @staticmethod
+    def combine(shared_partial: torch.Tensor | None, routed_out: torch.Tensor, group=None,
+                world_size: int = 1) -> torch.Tensor:
+        """bf16(all_reduce_sum(shared_partial) + routed_out): the caller's side
+        of the contract (``group``/``world_size`` of the tensor-parallel ranks;
+        no collective when world_size == 1)."""
+        if shared_partial is None:
+            return routed_out
+        if world_size > 1:
+            import torch.distributed as dist
+            dist.all_reduce(shared_partial, op=dist.ReduceOp.SUM, group=group)
+        return (shared_partial.float() + routed_out.float()).to(torch.bfloat16)

@@ -474,6 +474,26 @@ def dense_swiglu_mlp(x, w_gate_up, w_down):
     return expert_mlp(x, w_gate_up, w_down)
 
 
+def shared_expert_partial(x, w_gate_up, w_down, tp_size: int = 1, tp_rank: int = 0):
+    """Tensor-parallel rank ``tp_rank``'s partial output of the shared expert
+    (TileOPs PR #778, TP split convention and Partial output contract). The
+    complete weights are w_gate_up [2*F_s, H] (gate rows [0, F_s), up rows
+    [F_s, 2*F_s)) and w_down [H, F_s]; with F_p = F_s / tp_size the rank owns
+    gate rows [r*F_p, (r+1)*F_p), the up rows F_s above them (column
+    parallel) and w_down columns [r*F_p, (r+1)*F_p) (row parallel). The
+    partials of all ranks sum to the whole shared expert's output (float64)."""
+    two_fs = w_gate_up.shape[0]
+    F_s = two_fs // 2
+    if tp_size < 1 or not 0 <= tp_rank < tp_size or F_s % tp_size:
+        raise ValueError("need 0 <= tp_rank < tp_size and F_s % tp_size == 0")
+    Fp = F_s // tp_size
+    lo, hi = tp_rank * Fp, (tp_rank + 1) * Fp
+    gate = as_f64(w_gate_up[lo:hi])
+    up = as_f64(w_gate_up[F_s + lo:F_s + hi])
+    down = as_f64(w_down[:, lo:hi])
+    return dense_swiglu_mlp(x, np.concatenate([gate, up]), down)
+
+
 # ---------------------------------------------------------------------------
 # a7: weighted unpermute with routed_scaling_factor folded in
 # ---------------------------------------------------------------------------

@@ -1,0 +1,34 @@
+"""Worker of the world-size-2 gloo run in test_tp_gloo.py (spawned processes
+import it by module name)."""
+import datetime
+import os
+
+import numpy as np
+import torch
+import torch.distributed as dist
+
+
+def shared_contract_worker(rank: int, world: int, port: int, result_dir: str) -> None:
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        from moe_routed_expert_top_b200.layer import SharedFusedMoE
+        from oracle import moe_oracle as O
+        rng = np.random.default_rng(5)             # the same inputs on every rank
+        T, H, F_s = 6, 16, 16
+        bf = lambda a: torch.from_numpy(a.astype(np.float32)).to(torch.bfloat16)
+        x = bf(rng.standard_normal((T, H)))
+        wgu = bf(rng.standard_normal((2 * F_s, H)) * 0.3)
+        wd = bf(rng.standard_normal((H, F_s)) * 0.3)
+        routed = bf(rng.standard_normal((T, H)))
+        # this rank's partial (the GPU path's is checked against the same
+        # oracle partial rank by rank); combine all-reduces and adds
+        part = torch.from_numpy(O.shared_expert_partial(x, wgu, wd, world, rank)).float()
+        out = SharedFusedMoE.combine(part, routed, world_size=world)
+        full = O.dense_swiglu_mlp(x, wgu, wd)
+        assert np.allclose(part.numpy(), full, rtol=1e-5, atol=1e-5)   # reduced in place
+        ref = (torch.from_numpy(full).float() + routed.float()).to(torch.bfloat16).float()
+        assert torch.all((out.float() - ref).abs() <= ref.abs() * 2.0 ** -7 + 1e-6)
+        np.save(os.path.join(result_dir, f"rank{rank}.npy"), out.float().numpy())
+    finally:
+        dist.destroy_process_group()

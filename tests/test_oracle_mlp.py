@@ -87,6 +87,49 @@ def test_dense_reduction_to_textbook_swiglu_mlp():
         assert np.allclose(out[t], ref, rtol=1e-12, atol=1e-12)
 
 
+def _shard_token_loops(x, wgu, wd, F_s, tp, r):
+    """Scalar loops over rank r's FFN columns f in [r*F_s/tp, (r+1)*F_s/tp):
+    gate row f, up row F_s + f, down column f of the complete weights."""
+    Fp = F_s // tp
+    H = len(x)
+    y = [0.0] * H
+    for f in range(r * Fp, (r + 1) * Fp):
+        g = sum(float(x[i]) * float(wgu[f][i]) for i in range(H))
+        u = sum(float(x[i]) * float(wgu[F_s + f][i]) for i in range(H))
+        h = float(O.bf16_round(_silu(g) * u))
+        for n in range(H):
+            y[n] += h * float(wd[n][f])
+    return y
+
+
+@pytest.mark.parametrize("tp", [1, 2, 4])
+def test_shared_partial_brute_force_and_sum_of_shards(tp):
+    """Each rank's partial follows the pages' column/row-parallel split of the
+    complete weights (checked by scalar loops over the rank's columns), and the
+    partials of all ranks add up to the unsharded shared expert."""
+    rng = np.random.default_rng(40 + tp)
+    T, H, F_s = 3, 8, 8
+    x = _bf16(rng.standard_normal((T, H)))
+    wgu = _bf16(rng.standard_normal((2 * F_s, H)) * 0.3)
+    wd = _bf16(rng.standard_normal((H, F_s)) * 0.3)
+    xs, g, d = x.float().numpy(), wgu.float().numpy(), wd.float().numpy()
+    total = np.zeros((T, H))
+    for r in range(tp):
+        part = O.shared_expert_partial(x, wgu, wd, tp, r)
+        for t in range(T):
+            assert np.allclose(part[t], _shard_token_loops(xs[t], g, d, F_s, tp, r),
+                               rtol=1e-12, atol=1e-12)
+        total += part
+    full = O.dense_swiglu_mlp(x, wgu, wd)
+    assert np.allclose(total, full, rtol=1e-12, atol=1e-12)
+    for t in range(T):
+        assert np.allclose(full[t], _textbook_mlp_token(xs[t], g, d, F_s), rtol=1e-12, atol=1e-12)
+    with pytest.raises(ValueError):
+        O.shared_expert_partial(x, wgu, wd, 3, 0)      # F_s % tp != 0
+    with pytest.raises(ValueError):
+        O.shared_expert_partial(x, wgu, wd, tp, tp)    # rank out of range
+
+
 def test_brute_force_tiny_moe():
     rng = np.random.default_rng(2)
     T, E, k, H, F = 4, 3, 2, 8, 4
