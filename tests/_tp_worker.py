@@ -32,3 +32,22 @@ def shared_contract_worker(rank: int, world: int, port: int, result_dir: str) ->
         np.save(os.path.join(result_dir, f"rank{rank}.npy"), out.float().numpy())
     finally:
         dist.destroy_process_group()
+
+
+def bench_ranks_worker(rank: int, world: int, port: int, result_dir: str) -> None:
+    """bench.py's cross-rank steps on gloo: the barrier, the max over ranks of
+    a per-rank time, and the reference arm, which only rank 0 runs."""
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        import bench
+        bench.barrier(world)
+        got = bench.max_over_ranks(1.5 + rank, world, torch.device("cpu"))
+        assert got == 1.5 + (world - 1), got
+        if rank > 0:
+            os.environ["RANK"] = str(rank)
+            assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3"]) == 0
+        bench.barrier(world)
+        np.save(os.path.join(result_dir, f"bench{rank}.npy"), np.array([got]))
+    finally:
+        dist.destroy_process_group()
