@@ -402,6 +402,78 @@ def e4m3_value(codes) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
+# Training-side FP8 layouts and the SwiGLU backward (XTuner PR #2089,
+# §Changes: per_tile_quant_with_trans_per_block / _per_tile,
+# swiglu_per_tile_quant_with_trans_per_block, swiglu_backward)
+# ---------------------------------------------------------------------------
+
+
+def padded_columns(tables: dict) -> np.ndarray:
+    """Column of every row on the expert-padded token axis ("expand_128x"):
+    row r of expert g (rows go[g] .. go[g]+size[g]-1) goes to column
+    gpo[g] + (r - go[g]), i.e. each expert's rows start a fresh 128-row block
+    of the TileLang tutorial "Example 07" §1 layout (padding_M = 128)."""
+    sizes = np.asarray(tables["group_sizes"])
+    go = np.asarray(tables["group_offsets"])
+    gpo = np.asarray(tables["group_padded_offsets"])
+    cols = np.zeros(int(sizes.sum()), dtype=np.int64)
+    for g in range(len(sizes)):
+        n = int(sizes[g])
+        cols[go[g]:go[g] + n] = gpo[g] + np.arange(n)
+    return cols
+
+
+def quant_transposed(x32: np.ndarray, cols: np.ndarray, Mp: int, per_block: bool):
+    """The transposed, expert-padded FP8 copy of activations x [M, K] (the
+    operand of a weight-gradient GEMM, which contracts over tokens):
+    xT[k, cols[r]] = x[r, k], zero in the padding columns, xT [K, Mp]; then
+      per_block: one scale per 128x128 block of xT,
+      per tile : one scale per 1x128 tile of an xT row (128 padded tokens),
+    each with the rule of ``quant_1x128`` (s = amax/448, q = e4m3(x / s),
+    an all-zero block or tile has s = 0 and codes 0).
+    Returns qT uint8 [K, Mp] and sT float32 [K/128, Mp/128] or [K, Mp/128]."""
+    x = np.asarray(x32, dtype=np.float32)
+    M, K = x.shape
+    if K % 128 or Mp % 128:
+        raise ValueError("K and Mp must be multiples of 128")
+    xT = np.zeros((K, Mp), dtype=np.float32)
+    xT[:, cols] = x.T
+    if not per_block:
+        return quant_1x128(xT)
+    blocks = np.abs(xT).reshape(K // 128, 128, Mp // 128, 128)
+    amax = blocks.max(axis=(1, 3)).astype(np.float32)                  # [K/128, Mp/128]
+    s = (amax / F32(E4M3_MAX)).astype(np.float32)
+    s_full = np.repeat(np.repeat(s, 128, axis=0), 128, axis=1)
+    q = np.zeros((K, Mp), dtype=np.uint8)
+    nz = s_full > 0
+    q[nz] = e4m3_encode((xT[nz] / s_full[nz]).astype(np.float32))
+    return q, np.where(amax > 0, s, F32(0.0)).astype(np.float32)
+
+
+def quant_dual(x32: np.ndarray, cols: np.ndarray, Mp: int, per_block: bool):
+    """Both layouts of one activation: the forward 1x128 row quantisation
+    (``quant_1x128``) and the transposed, expert-padded copy
+    (``quant_transposed``). Returns (q, s, qT, sT)."""
+    q, s = quant_1x128(x32)
+    qT, sT = quant_transposed(x32, cols, Mp, per_block)
+    return q, s, qT, sT
+
+
+def swiglu_backward(gate_up, grad_h) -> np.ndarray:
+    """Gradient of h = SiLU(gate) * up with respect to [gate, up] given dL/dh,
+    float64: with s = 1 / (1 + e^-g),
+      dL/dgate = dL/dh * up * s * (1 + g * (1 - s))   (d SiLU/dg)
+      dL/dup   = dL/dh * g * s                        (SiLU(g))
+    Returns grad_gate_up [M, 2F] (gate columns first, as in gate_up)."""
+    G = as_f64(gate_up)
+    dh = as_f64(grad_h)
+    F = dh.shape[1]
+    g, u = G[:, :F], G[:, F:]
+    s = 1.0 / (1.0 + np.exp(-g))
+    return np.concatenate([dh * u * s * (1.0 + g * (1.0 - s)), dh * g * s], axis=1)
+
+
+# ---------------------------------------------------------------------------
 # a4 + a5 + a6: one expert's SwiGLU MLP on its rows
 # ---------------------------------------------------------------------------
 
