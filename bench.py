@@ -499,6 +499,90 @@ def run_reference(args, cfg) -> dict:
 
 
 # ---------------------------------------------------------------------------
+# single-op lines: the training-side FP8 kernels at the shapes of the
+# single-kernel benchmark of XTuner PR #2089 (x [131072, 6144] over 256
+# experts; gate_up [32768, 4096] and [131072, 8192] over 256 experts)
+# ---------------------------------------------------------------------------
+
+OPS = {
+    "quant_dual_block": dict(kind="dual", M=131072, K=6144, E=256, per_block=True),
+    "quant_dual_tile": dict(kind="dual", M=131072, K=6144, E=256, per_block=False),
+    "swiglu_quant_dual_32k": dict(kind="swiglu_dual", M=32768, K=2048, E=0, per_block=True),
+    "swiglu_quant_dual_128k": dict(kind="swiglu_dual", M=131072, K=4096, E=256, per_block=True),
+    "swiglu_backward_32k": dict(kind="backward", M=32768, K=2048),
+    "swiglu_backward_128k": dict(kind="backward", M=131072, K=4096),
+}
+OP_METRIC = "training-FP8 op ms + achieved GB/s, % of B200 HBM roofline (1 GPU)"
+
+
+def run_op(args, device) -> dict:
+    import moe_routed_expert_top_b200 as M
+    from moe_routed_expert_top_b200 import build
+    build.build()
+    spec = OPS[args.op]
+    kind, Mr, K = spec["kind"], spec["M"], spec["K"]
+    E = spec.get("E", 0)
+    g = torch.Generator(device=device)
+    g.manual_seed(7)
+    peaks = load_peaks()
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+    if kind == "backward":
+        gu = (torch.randn(Mr, 2 * K, generator=g, device=device) * 2).to(torch.bfloat16)
+        dh = torch.randn(Mr, K, generator=g, device=device).to(torch.bfloat16)
+        out = torch.empty(Mr, 2 * K, dtype=torch.bfloat16, device=device)
+        fn = lambda: M.moe_swiglu_backward(Mr, K, gu, dh, out)
+        nbytes = Mr * 2 * K * 2 + Mr * K * 2 + Mr * 2 * K * 2
+        shape = {"gate_up": [Mr, 2 * K]}
+    else:
+        prob, tables = None, None
+        if E:
+            # one expert per row, seeded uniform routing; tables from the library
+            ids = torch.from_numpy(np.random.default_rng(11).integers(0, E, size=(Mr, 1))
+                                   .astype(np.int32)).to(device)
+            prob = M.make_problem(T=Mr, H=128, F=128, E=E, top_k=1)
+            L = M.moe_get_tables_layout(prob)
+            tables = torch.empty(L["total_int32"], dtype=torch.int32, device=device)
+            st = torch.zeros(1, dtype=torch.int32, device=device)
+            M.moe_route_permute(prob, None, ids, None, None, None, tables, st)
+        M_blk = M.moe_dual_blocks(prob, Mr)
+        src_cols = 2 * K if kind == "swiglu_dual" else K
+        x = torch.randn(Mr, src_cols, generator=g, device=device).to(torch.bfloat16)
+        q = torch.empty(Mr, K, dtype=torch.uint8, device=device)
+        s = torch.empty(Mr, K // 128, device=device)
+        qT = torch.empty(K, 128 * M_blk, dtype=torch.uint8, device=device)
+        sT = torch.empty((K // 128, M_blk) if spec["per_block"] else (K, M_blk), device=device)
+        mode = M.MOE_TRANS_PER_BLOCK if spec["per_block"] else M.MOE_TRANS_PER_TILE
+        if kind == "swiglu_dual":
+            fn = lambda: M.moe_swiglu_quant_dual(prob, tables, Mr, K, x, mode, q, s, qT, sT)
+        else:
+            fn = lambda: M.moe_quant_dual(prob, tables, Mr, K, x, mode, q, s, qT, sT)
+        nbytes = (Mr * src_cols * 2 + Mr * K + s.numel() * 4 + qT.numel() + sT.numel() * 4)
+        shape = {"x" if kind == "dual" else "gate_up": [Mr, src_cols], "experts": E or 1,
+                 "trans": "per_block" if spec["per_block"] else "per_tile",
+                 "padded_tokens": 128 * M_blk}
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        times = time_steps(fn, args.steps, flush, stream)
+    ms = statistics.median(times)
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    return {
+        "metric": OP_METRIC, "op": args.op, "value": round(ms, 4), "unit": "ms",
+        "higher_is_better": False, "steps": args.steps, "warmup": args.warmup,
+        "dtype": "bf16 in, e4m3 + fp32 scales out" if kind != "backward" else "bf16",
+        "data": "synthetic", "config": {"workload": args.op, **shape,
+                                        "l2": "flushed (512 MiB write) before each call"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                     "traffic": None, "algorithmic_bytes": int(nbytes)},
+        "timing": "median of per-call CUDA events on the launching stream",
+        "clocks": clk.summary(),
+    }
+
+
+# ---------------------------------------------------------------------------
 # distributed plumbing
 # ---------------------------------------------------------------------------
 
@@ -530,8 +614,14 @@ def main(argv=None):
                     help="time eager calls instead of a CUDA graph replay of the forward")
     ap.add_argument("--override", default="",
                     help="workload fields to replace, e.g. E=16,T=256 (small profiling cases)")
+    ap.add_argument("--op", default=None, choices=list(OPS),
+                    help="time one training-side FP8 kernel instead of the forward (1 GPU)")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
+    if args.op is not None:
+        torch.cuda.set_device(0)
+        print(json.dumps(run_op(args, torch.device("cuda", 0))), flush=True)
+        return 0
     cfg = get_config(args.config)
     if args.override:
         kv = dict(item.split("=", 1) for item in args.override.split(","))

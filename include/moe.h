@@ -309,6 +309,50 @@ moe_status moe_shared_expert_forward(int32_t T, int32_t H, int32_t F_s, int32_t 
                                      const void* w_down, int32_t out_f32, void* out,
                                      void* workspace, size_t ws_bytes, moe_stream_t stream);
 
+/* ---- Training-side FP8 activation layouts (XTuner PR #2089 "Fuse MoE
+ * activation FP8 quantization kernels", Changes) --------------------------
+ *
+ * moe_quant_dual quantises an activation x bf16 [M, K] in one pass into
+ *   - the forward layout: q e4m3 [M, K], s fp32 [M, K/128] (one scale per
+ *     1x128 row tile; per_tile_quant), and
+ *   - a transposed, expert-padded copy for the weight-gradient GEMM:
+ *     qT e4m3 [K, 128*M_blk] where the rows of each expert start a fresh
+ *     128-token block (expand_128x): row r of expert g lands in column
+ *     group_padded_offsets[g] + (r - group_offsets[g]) (the block layout of
+ *     the TileLang tutorial "Example 07" section 1 with block_token 128);
+ *     padding columns are 0. Scales sT fp32 [K/128, M_blk] (trans_mode
+ *     MOE_TRANS_PER_BLOCK: one per 128x128 block) or [K, M_blk]
+ *     (MOE_TRANS_PER_TILE: one per 1x128 tile of a qT row).
+ * Scale rule: s = amax/448 (IEEE division), code = e4m3_rn_satfinite(x/s),
+ * all-zero tile/block: s = 0 and codes 0.
+ * Grouped mode: prob (padding_M 128) and `tables` from moe_route_permute,
+ * M == prob->T * prob->top_k, M_blk = the tables' M_blk. Dense mode (prob
+ * and tables NULL): one group, M_blk = ceil(M/128). Needs K % 128 == 0 and
+ * 16-byte-aligned pointers, else MOE_ERR_INVALID_ARG; M == 0 is a no-op.
+ * moe_dual_blocks returns M_blk (or -1 for invalid arguments). */
+enum { MOE_TRANS_PER_BLOCK = 0, MOE_TRANS_PER_TILE = 1 };
+int32_t moe_dual_blocks(const moe_problem* prob, int32_t M);
+moe_status moe_quant_dual(const moe_problem* prob, const int32_t* tables, int32_t M, int32_t K,
+                          const void* x, int32_t trans_mode, uint8_t* q, float* s, uint8_t* qT,
+                          float* sT, moe_stream_t stream);
+
+/* The same with x = SiLU(gate) * up computed in fp32 from gate_up bf16
+ * [M, 2F] (gate columns first) and never stored in bf16
+ * (swiglu_per_tile_quant_with_trans_per_block / _per_tile); K = F. debug_h,
+ * if not NULL, receives the fp32 h [M, F]. */
+moe_status moe_swiglu_quant_dual(const moe_problem* prob, const int32_t* tables, int32_t M,
+                                 int32_t F, const void* gate_up, int32_t trans_mode, uint8_t* q,
+                                 float* s, uint8_t* qT, float* sT, float* debug_h,
+                                 moe_stream_t stream);
+
+/* Backward of h = SiLU(gate) * up (swiglu_backward): from gate_up bf16
+ * [M, 2F] and grad_h bf16 [M, F], grad_gate_up bf16 [M, 2F] with
+ *   grad_gate = grad_h * up * s * (1 + g * (1 - s)),  grad_up = grad_h * g * s,
+ * s = 1 / (1 + e^-g), fp32 arithmetic. F % 8 == 0, 16-byte-aligned pointers,
+ * else MOE_ERR_INVALID_ARG; M == 0 is a no-op. */
+moe_status moe_swiglu_backward(int32_t M, int32_t F, const void* gate_up, const void* grad_h,
+                               void* grad_gate_up, moe_stream_t stream);
+
 /* Capacity of the library's built-in scratch area used by
  * moe_experts_forward_noalloc: 64 MiB of device memory. */
 #define MOE_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)

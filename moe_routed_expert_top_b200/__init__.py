@@ -19,6 +19,7 @@ __all__ = [
     "moe_grouped_gemm", "moe_swiglu_quant", "moe_unpermute", "moe_quantize_weight_128x128",
     "moe_experts_forward", "moe_decode_device_status", "moe_status_string",
     "moe_last_launch_count", "moe_shared_workspace_bytes", "moe_shared_expert_forward",
+    "moe_dual_blocks", "moe_quant_dual", "moe_swiglu_quant_dual", "moe_swiglu_backward",
     "EXPORTED_SYMBOLS",
     "MOE_OK", "MOE_EPI_STORE", "MOE_EPI_SWIGLU", "MOE_EPI_SWIGLU_FP8", "MOE_EPI_STORE_F32",
     "MOE_SCORE_SOFTMAX", "MOE_SCORE_SIGMOID", "MOE_DEV_BAD_EXPERT_ID", "MOE_DEV_TIMEOUT",
@@ -36,6 +37,7 @@ MOE_EPI_STORE, MOE_EPI_SWIGLU, MOE_EPI_SWIGLU_FP8, MOE_EPI_STORE_F32 = 0, 1, 2, 
 MOE_TILE_AUTO, MOE_TILE_TOKEN_ROWS, MOE_TILE_WEIGHT_ROWS = 0x00, 0x10, 0x20
 MOE_TILE_WEIGHT_ROWS_PAIR = 0x30
 MOE_A_GATHER = 0x100  # moe_grouped_gemm: A = hidden states, rows gathered through the tables
+MOE_TRANS_PER_BLOCK, MOE_TRANS_PER_TILE = 0, 1
 
 EXPORTED_SYMBOLS = (
     "moe_get_tables_layout", "moe_workspace_bytes", "moe_route_topk", "moe_route_permute",
@@ -43,6 +45,7 @@ EXPORTED_SYMBOLS = (
     "moe_experts_forward", "moe_decode_device_status", "moe_status_string",
     "moe_last_cuda_error", "moe_last_launch_count", "moe_experts_forward_noalloc",
     "moe_shared_workspace_bytes", "moe_shared_expert_forward",
+    "moe_dual_blocks", "moe_quant_dual", "moe_swiglu_quant_dual", "moe_swiglu_backward",
 )
 
 
@@ -121,6 +124,12 @@ def lib() -> ctypes.CDLL:
                                                                             ctypes.c_int32, _P,
                                                                             _P, ctypes.c_size_t,
                                                                             _P]),
+        "moe_dual_blocks": (ctypes.c_int32, [PP, ctypes.c_int32]),
+        "moe_quant_dual": (ctypes.c_int, [PP, _P, ctypes.c_int32, ctypes.c_int32, _P,
+                                          ctypes.c_int32, _P, _P, _P, _P, _P]),
+        "moe_swiglu_quant_dual": (ctypes.c_int, [PP, _P, ctypes.c_int32, ctypes.c_int32, _P,
+                                                 ctypes.c_int32, _P, _P, _P, _P, _P, _P]),
+        "moe_swiglu_backward": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, _P, _P, _P, _P]),
         "moe_decode_device_status": (ctypes.c_int, [ctypes.c_int32]),
         "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "moe_last_cuda_error": (ctypes.c_char_p, []),
@@ -239,6 +248,30 @@ def moe_shared_expert_forward(T, H, F_s, tp_size, tp_rank, hidden, w_gate_up, w_
                                            int(out_f32), _ptr(out), _ptr(workspace),
                                            int(ws_bytes), _stream(stream)),
            "moe_shared_expert_forward")
+
+
+def moe_dual_blocks(prob, M) -> int:
+    """128-token blocks of the padded token axis of moe_quant_dual (qT row pitch / 128)."""
+    return int(lib().moe_dual_blocks(ctypes.byref(prob) if prob is not None else None, int(M)))
+
+
+def moe_quant_dual(prob, tables, M, K, x, trans_mode, q, s, qT, sT, stream=None):
+    _check(lib().moe_quant_dual(ctypes.byref(prob) if prob is not None else None, _ptr(tables),
+                                int(M), int(K), _ptr(x), int(trans_mode), _ptr(q), _ptr(s),
+                                _ptr(qT), _ptr(sT), _stream(stream)), "moe_quant_dual")
+
+
+def moe_swiglu_quant_dual(prob, tables, M, F, gate_up, trans_mode, q, s, qT, sT, debug_h=None,
+                          stream=None):
+    _check(lib().moe_swiglu_quant_dual(ctypes.byref(prob) if prob is not None else None,
+                                       _ptr(tables), int(M), int(F), _ptr(gate_up),
+                                       int(trans_mode), _ptr(q), _ptr(s), _ptr(qT), _ptr(sT),
+                                       _ptr(debug_h), _stream(stream)), "moe_swiglu_quant_dual")
+
+
+def moe_swiglu_backward(M, F, gate_up, grad_h, grad_gate_up, stream=None):
+    _check(lib().moe_swiglu_backward(int(M), int(F), _ptr(gate_up), _ptr(grad_h),
+                                     _ptr(grad_gate_up), _stream(stream)), "moe_swiglu_backward")
 
 
 def moe_decode_device_status(dev_status: int) -> int:

@@ -20,9 +20,9 @@ BUILD_DIR = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmoe_b200.so")
 
 SOURCES = ["api.cu", "grouped_gemm.cu", "grouped_gemm_t.cu", "grouped_gemm_t2.cu",
-           "route_permute.cu", "tables.cu", "elementwise.cu", "no_alloc.cu"]
+           "route_permute.cu", "tables.cu", "elementwise.cu", "train_fp8.cu", "no_alloc.cu"]
 # translation units whose float32 results must not depend on FMA contraction
-NO_FMA = {"route_permute.cu", "elementwise.cu"}
+NO_FMA = {"route_permute.cu", "elementwise.cu", "train_fp8.cu"}
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xptxas", "-v",
          "-I", INCLUDE, "-I", CSRC]

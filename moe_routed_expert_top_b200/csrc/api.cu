@@ -480,6 +480,87 @@ moe_status moe_shared_expert_forward(int32_t T, int32_t H, int32_t F_s, int32_t 
   return MOE_OK;
 }
 
+int32_t moe_dual_blocks(const moe_problem* prob, int32_t M) {
+  if (M < 0) return -1;
+  if (prob == nullptr) return (M + 127) / 128;
+  if (check_problem(prob, false) != MOE_OK || prob->padding_M != 128) return -1;
+  if (static_cast<int64_t>(prob->T) * prob->top_k != M) return -1;
+  moe_tables_layout L;
+  fill_layout(prob, &L);
+  return L.M_blk;
+}
+
+namespace {
+
+moe_status quant_dual_common(const moe_problem* prob, const int32_t* tables, int32_t M,
+                             int32_t K, const void* x, int32_t trans_mode, uint8_t* q, float* s,
+                             uint8_t* qT, float* sT, float* debug_h, int swiglu,
+                             moe_stream_t stream) {
+  if ((prob == nullptr) != (tables == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (M < 0 || K <= 0 || K % 128 != 0) return MOE_ERR_INVALID_ARG;
+  if (trans_mode != MOE_TRANS_PER_BLOCK && trans_mode != MOE_TRANS_PER_TILE)
+    return MOE_ERR_INVALID_ARG;
+  const int32_t M_blk = moe_dual_blocks(prob, M);
+  if (M_blk < 0) return MOE_ERR_INVALID_ARG;
+  if (M == 0) return MOE_OK;
+  if (x == nullptr || q == nullptr || s == nullptr || qT == nullptr || sT == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(q) || !aligned16(qT) || (debug_h && !aligned16(debug_h)))
+    return MOE_ERR_INVALID_ARG;
+  moe::DualLaunch d;
+  d.M = M;
+  d.K = K;
+  d.M_blk = M_blk;
+  if (prob != nullptr) {
+    moe_tables_layout L;
+    fill_layout(prob, &L);
+    d.E = prob->E;
+    d.sizes = tables + L.group_sizes;
+    d.offsets = tables + L.group_offsets;
+    d.padded = tables + L.group_padded_offsets;
+    d.idx_for_bx = tables + L.group_idx_for_bx;
+  }
+  d.x = x;
+  d.swiglu = swiglu;
+  d.trans_block = trans_mode == MOE_TRANS_PER_BLOCK;
+  d.q = q;
+  d.s = s;
+  d.qT = qT;
+  d.sT = sT;
+  d.debug_h = debug_h;
+  MOE_CUDA_TRY(moe::launch_quant_dual(d, reinterpret_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+}  // namespace
+
+moe_status moe_quant_dual(const moe_problem* prob, const int32_t* tables, int32_t M, int32_t K,
+                          const void* x, int32_t trans_mode, uint8_t* q, float* s, uint8_t* qT,
+                          float* sT, moe_stream_t stream) {
+  return quant_dual_common(prob, tables, M, K, x, trans_mode, q, s, qT, sT, nullptr, 0, stream);
+}
+
+moe_status moe_swiglu_quant_dual(const moe_problem* prob, const int32_t* tables, int32_t M,
+                                 int32_t F, const void* gate_up, int32_t trans_mode, uint8_t* q,
+                                 float* s, uint8_t* qT, float* sT, float* debug_h,
+                                 moe_stream_t stream) {
+  return quant_dual_common(prob, tables, M, F, gate_up, trans_mode, q, s, qT, sT, debug_h, 1,
+                           stream);
+}
+
+moe_status moe_swiglu_backward(int32_t M, int32_t F, const void* gate_up, const void* grad_h,
+                               void* grad_gate_up, moe_stream_t stream) {
+  if (M < 0 || F <= 0 || F % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (M == 0) return MOE_OK;
+  if (gate_up == nullptr || grad_h == nullptr || grad_gate_up == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(gate_up) || !aligned16(grad_h) || !aligned16(grad_gate_up))
+    return MOE_ERR_INVALID_ARG;
+  MOE_CUDA_TRY(moe::launch_swiglu_backward(M, F, gate_up, grad_h, grad_gate_up,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
 moe_status moe_decode_device_status(int32_t dev_status) {
   if (dev_status == 0) return MOE_OK;
   if (dev_status & MOE_DEV_TIMEOUT) return MOE_ERR_TIMEOUT;

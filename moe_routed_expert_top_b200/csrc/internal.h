@@ -86,6 +86,29 @@ cudaError_t launch_swiglu_quant(int M, int F, const void* gate_up, const float* 
 cudaError_t launch_quantize_weight(int batch, int N, int K, const void* w, uint8_t* q,
                                    float* scales, cudaStream_t stream);
 
+// Training-side FP8 dual-layout quantisation (train_fp8.cu).
+struct DualLaunch {
+  int M = 0;  // rows of x
+  int K = 0;  // columns of the quantised activation (SwiGLU: F)
+  int E = 1;
+  const int32_t* sizes = nullptr;  // grouped mode (all four non-null) or dense (all null)
+  const int32_t* offsets = nullptr;
+  const int32_t* padded = nullptr;
+  const int32_t* idx_for_bx = nullptr;
+  int M_blk = 0;  // 128-token blocks of the padded axis (qT row pitch / 128)
+  const void* x = nullptr;  // bf16 [M, K], or gate_up bf16 [M, 2K] when swiglu
+  int swiglu = 0;
+  int trans_block = 1;  // 1: 128x128 block scales of xT; 0: 1x128 tile scales
+  uint8_t* q = nullptr;
+  float* s = nullptr;
+  uint8_t* qT = nullptr;
+  float* sT = nullptr;
+  float* debug_h = nullptr;
+};
+cudaError_t launch_quant_dual(const DualLaunch& L, cudaStream_t stream);
+cudaError_t launch_swiglu_backward(int M, int F, const void* gate_up, const void* grad_h,
+                                   void* grad_gate_up, cudaStream_t stream);
+
 // Streaming multiprocessors of the current device (cached per device).
 int device_sm_count();
 
