@@ -519,7 +519,13 @@ def run_op(args, device) -> dict:
     import moe_routed_expert_top_b200 as M
     from moe_routed_expert_top_b200 import build
     build.build()
-    spec = OPS[args.op]
+    spec = dict(OPS[args.op])
+    if args.override:       # e.g. M=32768: a smaller case of the same op (profiling)
+        for item in args.override.split(","):
+            key, val = item.split("=", 1)
+            if key not in ("M", "K"):
+                raise SystemExit(f"--override for --op takes M and K, not {key}")
+            spec[key] = int(val)
     kind, Mr, K = spec["kind"], spec["M"], spec["K"]
     E = spec.get("E", 0)
     g = torch.Generator(device=device)

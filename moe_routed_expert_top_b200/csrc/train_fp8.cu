@@ -35,7 +35,7 @@ namespace {
 constexpr int kTileStride = 129;
 constexpr int kTileStrideBf16 = 136;
 __host__ __device__ constexpr int dual_smem(bool swiglu) {
-  return (swiglu ? 128 * kTileStride * 4 : 128 * kTileStrideBf16 * 2) + 256 * 4;
+  return (swiglu ? 128 * kTileStride * 4 : 128 * kTileStrideBf16 * 2) + 512 * 4;  // + reduce
 }
 
 struct DualParams {
@@ -83,13 +83,13 @@ __device__ __forceinline__ float div_by_scale(float x, float s, float y) {
 
 constexpr float kFastDivMinScale = 8.0779356e-28f;  // 2^-90
 
-// 64 values -> 64 E4M3 codes (scale s, or all zero when amax == 0) as 4 x 16 B.
-__device__ __forceinline__ void encode64(const float* v, float amax, float s, uint4* out) {
-  uint32_t w[16];
+// 32 values -> 32 E4M3 codes (scale s, or all zero when amax == 0) as 2 x 16 B.
+__device__ __forceinline__ void encode32(const float* v, float amax, float s, uint4* out) {
+  uint32_t w[8];
   if (amax > 0.0f && s >= kFastDivMinScale) {
     const float y = __frcp_rn(s);
 #pragma unroll
-    for (int j = 0; j < 16; ++j)
+    for (int j = 0; j < 8; ++j)
       w[j] = static_cast<uint32_t>(cvt_e4m3x2(div_by_scale(v[4 * j], s, y),
                                               div_by_scale(v[4 * j + 1], s, y))) |
              (static_cast<uint32_t>(cvt_e4m3x2(div_by_scale(v[4 * j + 2], s, y),
@@ -97,29 +97,32 @@ __device__ __forceinline__ void encode64(const float* v, float amax, float s, ui
               << 16);
   } else if (amax > 0.0f) {
 #pragma unroll
-    for (int j = 0; j < 16; ++j)
+    for (int j = 0; j < 8; ++j)
       w[j] = static_cast<uint32_t>(cvt_e4m3x2(v[4 * j] / s, v[4 * j + 1] / s)) |
              (static_cast<uint32_t>(cvt_e4m3x2(v[4 * j + 2] / s, v[4 * j + 3] / s)) << 16);
   } else {
 #pragma unroll
-    for (int j = 0; j < 16; ++j) w[j] = 0u;
+    for (int j = 0; j < 8; ++j) w[j] = 0u;
   }
-#pragma unroll
-  for (int j = 0; j < 4; ++j) out[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+  out[0] = make_uint4(w[0], w[1], w[2], w[3]);
+  out[1] = make_uint4(w[4], w[5], w[6], w[7]);
 }
 
+constexpr int kDualThreads = 512;
+
 // One CTA per (128-token block bx of the padded axis, 128-column block kb);
-// 256 threads. Phase A: thread (row i = t/2, half t%2) reads 64 values of its
-// row, writes the row-layout codes and scale (each row segment is one 1x128
-// tile) and stages the values in shared memory. Phase B: thread (column
-// c = t%128, token half t/128) reads 64 staged values down its column and
-// writes them as 64 contiguous codes of xT row kb*128 + c.
+// 512 threads, 32 values each. Phase A: thread (row i = t/4, quarter t%4)
+// reads 32 values of its row, writes their row-layout codes (each row segment
+// of 128 is one 1x128 tile, its amax shared by the row's 4 threads) and stages
+// the values in shared memory. Phase B: thread (column c = t%128, token
+// quarter t/128) reads 32 staged values down its column and writes them as 32
+// contiguous codes of xT row kb*128 + c.
 template <bool kSwiglu, bool kTransBlock>
-__global__ void __launch_bounds__(256) quant_dual_kernel(const DualParams p) {
+__global__ void __launch_bounds__(kDualThreads, 2) quant_dual_kernel(const DualParams p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   float* tile = reinterpret_cast<float*>(smem_raw);                  // SwiGLU: [128][129] fp32
   __nv_bfloat16* tile16 = reinterpret_cast<__nv_bfloat16*>(smem_raw);  // plain: [128][136] bf16
-  float* red = reinterpret_cast<float*>(smem_raw + dual_smem(kSwiglu) - 256 * 4);  // [256]
+  float* red = reinterpret_cast<float*>(smem_raw + dual_smem(kSwiglu) - kDualThreads * 4);
   const int bx = blockIdx.x;
   const int kb = blockIdx.y;
   const int t = threadIdx.x;
@@ -142,85 +145,92 @@ __global__ void __launch_bounds__(256) quant_dual_kernel(const DualParams p) {
 
   // ---------------------------------------------------------------- phase A
   {
-    const int i = t >> 1;
-    const int hh = t & 1;
-    const int col = kb * 128 + hh * 64;
-    float v[64];
+    const int i = t >> 2;
+    const int qq = t & 3;
+    const int col = kb * 128 + qq * 32;
+    float v[32];
     const bool live = i < rows;
     if (live) {
       const int64_t r = static_cast<int64_t>(m_start + i);
       if constexpr (kSwiglu) {
         const uint4* gsrc = reinterpret_cast<const uint4*>(p.x + r * 2 * p.K + col);
         const uint4* usrc = reinterpret_cast<const uint4*>(p.x + r * 2 * p.K + p.K + col);
+        uint4 graw[4], uraw[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 4; ++j) {
+          graw[j] = __ldg(gsrc + j);
+          uraw[j] = __ldg(usrc + j);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
           float g[8], u[8];
-          unpack8(__ldg(gsrc + j), g);
-          unpack8(__ldg(usrc + j), u);
+          unpack8(graw[j], g);
+          unpack8(uraw[j], u);
 #pragma unroll
           for (int e = 0; e < 8; ++e) v[8 * j + e] = g[e] / (1.0f + expf(-g[e])) * u[e];
         }
       } else {
         const uint4* src = reinterpret_cast<const uint4*>(p.x + r * p.K + col);
-        uint4 raw[8];
+        uint4 raw[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) raw[j] = __ldg(src + j);
-        uint4* st = reinterpret_cast<uint4*>(tile16 + i * kTileStrideBf16 + hh * 64);
+        for (int j = 0; j < 4; ++j) raw[j] = __ldg(src + j);
+        uint4* st = reinterpret_cast<uint4*>(tile16 + i * kTileStrideBf16 + qq * 32);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 4; ++j) {
           st[j] = raw[j];
           unpack8(raw[j], v + 8 * j);
         }
       }
     } else {
 #pragma unroll
-      for (int j = 0; j < 64; ++j) v[j] = 0.0f;
+      for (int j = 0; j < 32; ++j) v[j] = 0.0f;
       if constexpr (!kSwiglu) {
-        uint4* st = reinterpret_cast<uint4*>(tile16 + i * kTileStrideBf16 + hh * 64);
+        uint4* st = reinterpret_cast<uint4*>(tile16 + i * kTileStrideBf16 + qq * 32);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) st[j] = make_uint4(0u, 0u, 0u, 0u);
+        for (int j = 0; j < 4; ++j) st[j] = make_uint4(0u, 0u, 0u, 0u);
       }
     }
     float amax = 0.0f;
 #pragma unroll
-    for (int j = 0; j < 64; ++j) amax = fmaxf(amax, fabsf(v[j]));
+    for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(v[j]));
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
     const float s = amax / 448.0f;
     if (live) {
       const int64_t r = static_cast<int64_t>(m_start + i);
-      uint4 codes[4];
-      encode64(v, amax, s, codes);
+      uint4 codes[2];
+      encode32(v, amax, s, codes);
       uint4* dst = reinterpret_cast<uint4*>(p.q + r * p.K + col);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) dst[j] = codes[j];
-      if (hh == 0) p.s[r * KB + kb] = amax > 0.0f ? s : 0.0f;
+      dst[0] = codes[0];
+      dst[1] = codes[1];
+      if (qq == 0) p.s[r * KB + kb] = amax > 0.0f ? s : 0.0f;
       if (kSwiglu && p.debug_h != nullptr) {
         float4* hd = reinterpret_cast<float4*>(p.debug_h + r * p.K + col);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) hd[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        for (int j = 0; j < 8; ++j) hd[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
       }
     }
     if constexpr (kSwiglu) {
 #pragma unroll
-      for (int j = 0; j < 64; ++j) tile[i * kTileStride + hh * 64 + j] = v[j];
+      for (int j = 0; j < 32; ++j) tile[i * kTileStride + qq * 32 + j] = v[j];
     }
   }
   __syncthreads();
 
   // ---------------------------------------------------------------- phase B
   const int c = t & 127;
-  const int th = t >> 7;
-  float w[64];
+  const int tq = t >> 7;
+  float w[32];
   if constexpr (kSwiglu) {
 #pragma unroll
-    for (int r = 0; r < 64; ++r) w[r] = tile[(th * 64 + r) * kTileStride + c];
+    for (int r = 0; r < 32; ++r) w[r] = tile[(tq * 32 + r) * kTileStride + c];
   } else {
 #pragma unroll
-    for (int r = 0; r < 64; ++r) w[r] = __bfloat162float(tile16[(th * 64 + r) * kTileStrideBf16 + c]);
+    for (int r = 0; r < 32; ++r) w[r] = __bfloat162float(tile16[(tq * 32 + r) * kTileStrideBf16 + c]);
   }
   float amax = 0.0f;
 #pragma unroll
-  for (int r = 0; r < 64; ++r) amax = fmaxf(amax, fabsf(w[r]));
+  for (int r = 0; r < 32; ++r) amax = fmaxf(amax, fabsf(w[r]));
   if constexpr (kTransBlock) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
@@ -228,25 +238,25 @@ __global__ void __launch_bounds__(256) quant_dual_kernel(const DualParams p) {
     __syncthreads();
     amax = red[0];
 #pragma unroll
-    for (int wi = 1; wi < 8; ++wi) amax = fmaxf(amax, red[wi]);
+    for (int wi = 1; wi < kDualThreads / 32; ++wi) amax = fmaxf(amax, red[wi]);
   } else {
     red[t] = amax;
     __syncthreads();
-    amax = fmaxf(red[c], red[c + 128]);
+    amax = fmaxf(fmaxf(red[c], red[c + 128]), fmaxf(red[c + 256], red[c + 384]));
   }
   const float s = amax / 448.0f;
-  uint4 codes[4];
-  encode64(w, amax, s, codes);
+  uint4 codes[2];
+  encode32(w, amax, s, codes);
   const int64_t ldT = static_cast<int64_t>(p.M_blk) * 128;
   uint4* dst = reinterpret_cast<uint4*>(p.qT + static_cast<int64_t>(kb * 128 + c) * ldT +
-                                        static_cast<int64_t>(bx) * 128 + th * 64);
-#pragma unroll
-  for (int j = 0; j < 4; ++j) dst[j] = codes[j];
+                                        static_cast<int64_t>(bx) * 128 + tq * 32);
+  dst[0] = codes[0];
+  dst[1] = codes[1];
   const float sv = amax > 0.0f ? s : 0.0f;
   if constexpr (kTransBlock) {
     if (t == 0) p.sT[static_cast<int64_t>(kb) * p.M_blk + bx] = sv;
   } else {
-    if (th == 0) p.sT[static_cast<int64_t>(kb * 128 + c) * p.M_blk + bx] = sv;
+    if (tq == 0) p.sT[static_cast<int64_t>(kb * 128 + c) * p.M_blk + bx] = sv;
   }
 }
 
@@ -296,7 +306,7 @@ cudaError_t run_dual(const DualParams& p, cudaStream_t stream) {
     attr_done[dev] = true;
   }
   const dim3 grid(static_cast<unsigned>(p.M_blk), static_cast<unsigned>(p.K / 128));
-  quant_dual_kernel<kSwiglu, kTransBlock><<<grid, 256, dual_smem(kSwiglu), stream>>>(p);
+  quant_dual_kernel<kSwiglu, kTransBlock><<<grid, kDualThreads, dual_smem(kSwiglu), stream>>>(p);
   return cudaGetLastError();
 }
 
