@@ -40,29 +40,35 @@ PAGE_MS = {"qwen3_decode": 3.219, "qwen3_prefill": 6.778, "dsv3_decode_fp8": Non
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-def csrc_sha256() -> str:
-    """Hash of the CUDA sources: a recorded ncu traffic figure is only valid for
-    the exact kernels it was measured on."""
+def sources_sha256(files) -> str:
+    """Hash of the named CUDA source files (paths relative to the package's
+    csrc/): a recorded ncu traffic figure is only valid for the exact kernel
+    sources it was measured on."""
     import hashlib
     d = os.path.join(ROOT, "moe_routed_expert_top_b200", "csrc")
     h = hashlib.sha256()
-    for f in sorted(os.listdir(d)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            h.update(f.encode())
-            h.update(open(os.path.join(d, f), "rb").read())
+    for f in sorted(files):
+        h.update(f.encode())
+        h.update(open(os.path.join(d, f), "rb").read())
     return h.hexdigest()
 
 
 def recorded_traffic(workload: str, kernel: str):
     """DRAM bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)
     recorded in profiles/roofline_traffic.json for this workload's dominant
-    kernel, or None if absent or taken on different kernel sources."""
+    kernel, or None if absent or if any source file of that kernel (listed in
+    the record) changed since."""
     p = os.path.join(ROOT, "profiles", "roofline_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         rec = json.load(f).get(workload)
-    if not rec or rec.get("kernel") != kernel or rec.get("source_sha256") != csrc_sha256():
+    if not rec or rec.get("kernel") != kernel or not rec.get("sources"):
+        return None
+    try:
+        if rec.get("source_sha256") != sources_sha256(rec["sources"]):
+            return None
+    except OSError:
         return None
     return rec.get("traffic_bytes")
 
