@@ -139,7 +139,10 @@ typedef struct moe_problem {
   int32_t H;            /* hidden size: multiple of 64 (of 128 with down_fp8) */
   int32_t F;            /* expert FFN size: multiple of 64 (of 128 with down_fp8) */
   int32_t E;            /* routed experts, 1..1024 */
-  int32_t top_k;        /* 1..min(E, 32) */
+  int32_t top_k;        /* 1..32; at most E for routing and the forward (k distinct
+                           experts); tables, GEMMs and unpermute over given ids
+                           accept repeated groups (e.g. the ranks of expert
+                           parallelism) */
   int32_t padding_M;    /* group_padded_offsets alignment = M-block height
                            ("block_token" in [TUT07]); the GEMMs need 128 */
   int32_t score_fn;     /* MOE_SCORE_SOFTMAX or MOE_SCORE_SIGMOID */
@@ -352,6 +355,27 @@ moe_status moe_swiglu_quant_dual(const moe_problem* prob, const int32_t* tables,
  * else MOE_ERR_INVALID_ARG; M == 0 is a no-op. */
 moe_status moe_swiglu_backward(int32_t M, int32_t F, const void* gate_up, const void* grad_h,
                                void* grad_gate_up, moe_stream_t stream);
+
+/* ---- Expert parallelism helpers (experts split over `world` ranks of
+ * E_local experts each; pypto-lib PR #809 "predicate empty routed-expert
+ * stages": dispatch to the ranks owning the experts, per-rank expert counts,
+ * empty local experts skipped). The exchange itself is the caller's
+ * all-to-all; the rest of the path is the entry points above. -------------
+ *
+ * moe_ep_split_ids: for n expert ids, rank_ids[i] = id / E_local and
+ * local_ids[i] = id % E_local; an id outside [0, world*E_local) gets rank
+ * `world` (flagged by moe_route_permute as a bad id when the ranks are used
+ * as its groups) and local id 0. n < 0, E_local < 1, world < 1 or null
+ * pointers -> MOE_ERR_INVALID_ARG; n == 0 is a no-op. */
+moe_status moe_ep_split_ids(int32_t n, int32_t E_local, int32_t world, const int32_t* ids,
+                            int32_t* rank_ids, int32_t* local_ids, moe_stream_t stream);
+
+/* moe_gather_rows: dst row r = src row map[r] for n_dst rows of row_bytes
+ * bytes (a multiple of 4); map[r] < 0 gives a zero row; map[r] >= n_src gives
+ * a zero row and ORs MOE_DEV_BAD_TABLES into *dev_status (if not NULL).
+ * Caller-owned device memory; rows do not overlap between src and dst. */
+moe_status moe_gather_rows(int32_t n_dst, int32_t n_src, int64_t row_bytes, const int32_t* map,
+                           const void* src, void* dst, int32_t* dev_status, moe_stream_t stream);
 
 /* Capacity of the library's built-in scratch area used by
  * moe_experts_forward_noalloc: 64 MiB of device memory. */

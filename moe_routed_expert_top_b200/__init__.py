@@ -20,7 +20,7 @@ __all__ = [
     "moe_experts_forward", "moe_decode_device_status", "moe_status_string",
     "moe_last_launch_count", "moe_shared_workspace_bytes", "moe_shared_expert_forward",
     "moe_dual_blocks", "moe_quant_dual", "moe_swiglu_quant_dual", "moe_swiglu_backward",
-    "EXPORTED_SYMBOLS",
+    "moe_ep_split_ids", "moe_gather_rows", "EXPORTED_SYMBOLS",
     "MOE_OK", "MOE_EPI_STORE", "MOE_EPI_SWIGLU", "MOE_EPI_SWIGLU_FP8", "MOE_EPI_STORE_F32",
     "MOE_SCORE_SOFTMAX", "MOE_SCORE_SIGMOID", "MOE_DEV_BAD_EXPERT_ID", "MOE_DEV_TIMEOUT",
 ]
@@ -46,6 +46,7 @@ EXPORTED_SYMBOLS = (
     "moe_last_cuda_error", "moe_last_launch_count", "moe_experts_forward_noalloc",
     "moe_shared_workspace_bytes", "moe_shared_expert_forward",
     "moe_dual_blocks", "moe_quant_dual", "moe_swiglu_quant_dual", "moe_swiglu_backward",
+    "moe_ep_split_ids", "moe_gather_rows",
 )
 
 
@@ -130,6 +131,10 @@ def lib() -> ctypes.CDLL:
         "moe_swiglu_quant_dual": (ctypes.c_int, [PP, _P, ctypes.c_int32, ctypes.c_int32, _P,
                                                  ctypes.c_int32, _P, _P, _P, _P, _P, _P]),
         "moe_swiglu_backward": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, _P, _P, _P, _P]),
+        "moe_ep_split_ids": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _P,
+                                            _P, _P, _P]),
+        "moe_gather_rows": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int64, _P, _P,
+                                           _P, _P, _P]),
         "moe_decode_device_status": (ctypes.c_int, [ctypes.c_int32]),
         "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "moe_last_cuda_error": (ctypes.c_char_p, []),
@@ -272,6 +277,16 @@ def moe_swiglu_quant_dual(prob, tables, M, F, gate_up, trans_mode, q, s, qT, sT,
 def moe_swiglu_backward(M, F, gate_up, grad_h, grad_gate_up, stream=None):
     _check(lib().moe_swiglu_backward(int(M), int(F), _ptr(gate_up), _ptr(grad_h),
                                      _ptr(grad_gate_up), _stream(stream)), "moe_swiglu_backward")
+
+
+def moe_ep_split_ids(n, E_local, world, ids, rank_ids, local_ids, stream=None):
+    _check(lib().moe_ep_split_ids(int(n), int(E_local), int(world), _ptr(ids), _ptr(rank_ids),
+                                  _ptr(local_ids), _stream(stream)), "moe_ep_split_ids")
+
+
+def moe_gather_rows(n_dst, n_src, row_bytes, map_, src, dst, dev_status=None, stream=None):
+    _check(lib().moe_gather_rows(int(n_dst), int(n_src), int(row_bytes), _ptr(map_), _ptr(src),
+                                 _ptr(dst), _ptr(dev_status), _stream(stream)), "moe_gather_rows")
 
 
 def moe_decode_device_status(dev_status: int) -> int:

@@ -39,10 +39,13 @@ moe_status check_problem(const moe_problem* pr, bool need_gemm) {
     return MOE_ERR_INVALID_ARG;
   if (pr->score_fn != MOE_SCORE_SOFTMAX && pr->score_fn != MOE_SCORE_SIGMOID)
     return MOE_ERR_INVALID_ARG;
-  if (pr->E > 1024 || pr->top_k > 32 || pr->top_k > pr->E) return MOE_ERR_UNSUPPORTED;
+  if (pr->E > 1024 || pr->top_k > 32) return MOE_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(pr->T) * pr->top_k > kMaxPairs) return MOE_ERR_UNSUPPORTED;
   if (pr->padding_M > (1 << 20)) return MOE_ERR_UNSUPPORTED;
   if (need_gemm) {
+    // a token's k experts are distinct; tables over given ids accept repeats
+    // (the groups can be ranks, as in expert parallelism)
+    if (pr->top_k > pr->E) return MOE_ERR_UNSUPPORTED;
     if (pr->padding_M != 128) return MOE_ERR_UNSUPPORTED;
     if (pr->H % 64 != 0 || pr->F % 64 != 0 || pr->F_shared % 64 != 0) return MOE_ERR_UNSUPPORTED;
     if (pr->down_fp8 && (pr->H % 128 != 0 || pr->F % 128 != 0)) return MOE_ERR_UNSUPPORTED;
@@ -124,6 +127,7 @@ moe_status moe_route_topk(const moe_problem* prob, const float* logits, int32_t*
                           float* topk_weights, moe_stream_t stream) {
   moe_status s = check_problem(prob, false);
   if (s != MOE_OK) return s;
+  if (prob->top_k > prob->E) return MOE_ERR_UNSUPPORTED;  // k distinct experts
   if (prob->T == 0) return MOE_OK;
   if (logits == nullptr || topk_ids == nullptr || topk_weights == nullptr)
     return MOE_ERR_INVALID_ARG;
@@ -138,6 +142,7 @@ moe_status moe_route_permute(const moe_problem* prob, const float* logits, int32
                              int32_t* tables, int32_t* dev_status, moe_stream_t stream) {
   moe_status s = check_problem(prob, false);
   if (s != MOE_OK) return s;
+  if (logits != nullptr && prob->top_k > prob->E) return MOE_ERR_UNSUPPORTED;
   if (prob->T == 0) return MOE_OK;
   if (topk_ids == nullptr || tables == nullptr || dev_status == nullptr)
     return MOE_ERR_INVALID_ARG;
@@ -557,6 +562,30 @@ moe_status moe_swiglu_backward(int32_t M, int32_t F, const void* gate_up, const 
   if (!aligned16(gate_up) || !aligned16(grad_h) || !aligned16(grad_gate_up))
     return MOE_ERR_INVALID_ARG;
   MOE_CUDA_TRY(moe::launch_swiglu_backward(M, F, gate_up, grad_h, grad_gate_up,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_ep_split_ids(int32_t n, int32_t E_local, int32_t world, const int32_t* ids,
+                            int32_t* rank_ids, int32_t* local_ids, moe_stream_t stream) {
+  if (n < 0 || E_local < 1 || world < 1) return MOE_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(E_local) * world > (1ll << 30)) return MOE_ERR_INVALID_ARG;
+  if (n == 0) return MOE_OK;
+  if (ids == nullptr || rank_ids == nullptr || local_ids == nullptr) return MOE_ERR_INVALID_ARG;
+  MOE_CUDA_TRY(moe::launch_split_ids(n, E_local, world, ids, rank_ids, local_ids,
+                                     reinterpret_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_gather_rows(int32_t n_dst, int32_t n_src, int64_t row_bytes, const int32_t* map,
+                           const void* src, void* dst, int32_t* dev_status, moe_stream_t stream) {
+  if (n_dst < 0 || n_src < 0 || row_bytes <= 0 || row_bytes % 4 != 0) return MOE_ERR_INVALID_ARG;
+  if (row_bytes / 4 > (1ll << 30)) return MOE_ERR_INVALID_ARG;
+  if (n_dst == 0) return MOE_OK;
+  if (map == nullptr || dst == nullptr || (n_src > 0 && src == nullptr)) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(dst) & 3) != 0 || (reinterpret_cast<uintptr_t>(src) & 3) != 0)
+    return MOE_ERR_INVALID_ARG;
+  MOE_CUDA_TRY(moe::launch_gather_rows_any(n_dst, n_src, row_bytes, map, src, dst, dev_status,
                                            reinterpret_cast<cudaStream_t>(stream)));
   return MOE_OK;
 }

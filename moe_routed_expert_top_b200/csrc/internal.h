@@ -109,6 +109,13 @@ cudaError_t launch_quant_dual(const DualLaunch& L, cudaStream_t stream);
 cudaError_t launch_swiglu_backward(int M, int F, const void* gate_up, const void* grad_h,
                                    void* grad_gate_up, cudaStream_t stream);
 
+// Expert parallelism helpers (ep.cu).
+cudaError_t launch_split_ids(int n, int E_local, int world, const int32_t* ids, int32_t* rank_ids,
+                             int32_t* local_ids, cudaStream_t stream);
+cudaError_t launch_gather_rows_any(int n_dst, int n_src, long long row_bytes, const int32_t* map,
+                                   const void* src, void* dst, int32_t* status,
+                                   cudaStream_t stream);
+
 // Streaming multiprocessors of the current device (cached per device).
 int device_sm_count();
 

@@ -51,3 +51,27 @@ def bench_ranks_worker(rank: int, world: int, port: int, result_dir: str) -> Non
         np.save(os.path.join(result_dir, f"bench{rank}.npy"), np.array([got]))
     finally:
         dist.destroy_process_group()
+
+
+def ep_exchange_worker(rank: int, world: int, port: int, result_dir: str) -> None:
+    """ep.TorchDistExchange on gloo: counts, uneven row splits (one empty),
+    and the reverse exchange bringing every row back to its sender in order."""
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        from moe_routed_expert_top_b200.ep import TorchDistExchange
+        ex = TorchDistExchange()
+        send_counts = torch.tensor([[2, 3], [0, 4]][rank], dtype=torch.int32)
+        # row value = 100*source + position in the source's send buffer
+        send = torch.stack([torch.full((3,), 100.0 * rank + i) for i in range(int(send_counts.sum()))])
+        ss, rs = ex.counts(send_counts)
+        assert ss == send_counts.tolist()
+        assert rs == [[2, 0], [3, 4]][rank]
+        recv = ex.rows(send, ss, rs)
+        want = {0: [0, 1], 1: [2, 3, 4, 100, 101, 102, 103]}[rank]
+        assert recv[:, 0].tolist() == [float(v) for v in want]
+        back = ex.rows(recv * 2, rs, ss)                       # the reverse direction
+        assert torch.equal(back, send * 2)
+        np.save(os.path.join(result_dir, f"ep{rank}.npy"), back.numpy())
+    finally:
+        dist.destroy_process_group()
