@@ -334,6 +334,15 @@ def run_b200(args, cfg, rank, world, device):
     # stage breakdown and the dominant kernel's roofline
     stages = stage_breakdown(M, layer, cfg, hidden, ids, weights, max(5, min(args.steps, 30)),
                              flush)
+    # top-k routing from the router logits (a1), timed on its own: the forward
+    # takes the routing as input
+    r_ids = torch.empty_like(ids)
+    r_w = torch.empty_like(weights)
+    prob_r = layer.problem(cfg.T)
+    route = lambda: M.moe_route_topk(prob_r, logits, r_ids, r_w)
+    for _ in range(3):
+        route()
+    routing_ms = statistics.median(time_steps(route, max(5, min(args.steps, 30)), flush, stream))
     dom = max(("gate_up_gemm", "down_gemm"), key=lambda s: stages[s])
     dom_bytes = wm["gate_up_bytes"] if dom == "gate_up_gemm" else wm["down_bytes"]
     dom_flops = wm["gate_up_flops"] if dom == "gate_up_gemm" else wm["down_flops"]
@@ -379,6 +388,8 @@ def run_b200(args, cfg, rank, world, device):
                    "parallelism": f"replicas x{world}"},
         "roofline": roof, "forward_roofline": fwd_roof,
         "stages_ms": {k: round(v, 4) for k, v in stages.items()},
+        "routing_ms": round(routing_ms, 4),
+        "tflops_routed": round(world * wm["flops_routed"] / t_s / 1e12, 2),
         "launch": "cuda graph replay of moe_experts_forward" if not args.no_graph
                   else "eager moe_experts_forward calls",
         "eager_ms": round(eager_ms, 4),
