@@ -113,8 +113,10 @@ __device__ __forceinline__ bool p_decode(const PParams& p, const int* cpre, int 
   ti.e = e;
   ti.wb = wb;
   ti.chunks = chunks;
-  ti.m0 = off + c * TN;
-  ti.nt = pmin(TN, size - c * TN);
+  // the expert's tokens split evenly over its tiles (in multiples of 32)
+  const int ts = pmin(TN, ((size + chunks - 1) / chunks + 31) & ~31);
+  ti.m0 = off + c * ts;
+  ti.nt = pmin(ts, size - c * ts);
   if (ti.nt <= 0 || ti.m0 < 0 || ti.m0 + ti.nt > p.rows_total) {
     if (threadIdx.x == 0 && ti.nt > 0) atomicOr(p.status, MOE_DEV_BAD_TABLES_FLAG);
     return false;

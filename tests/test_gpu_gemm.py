@@ -66,6 +66,10 @@ GEMM_CASES = [
     (300, 5, 1, 192, 256, [0, 0, 300, 0, 0]),
     # more tiles than resident CTAs: every persistent loop wraps
     (2048, 16, 4, 512, 512, None),
+    # experts just past one or two token tiles (the pair tiling splits them
+    # evenly over their tiles): 256-token tiles, then 64-token ones
+    (546, 8, 4, 256, 256, [257, 288, 289, 517, 544, 256, 0, 33]),
+    (256, 8, 2, 256, 256, [65, 96, 97, 160, 64, 0, 1, 29]),
 ]
 
 
