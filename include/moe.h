@@ -261,6 +261,37 @@ moe_status moe_unpermute(const moe_problem* prob, const float* y, const int32_t*
                          const float* topk_weights, float scale, const float* addend,
                          void* out, moe_stream_t stream);
 
+/* a6 with the routing weight folded into the epilogue ([PR1580] Unpermute's
+ * scale folding, applied one step earlier, as the down projection's per-row
+ * scale × routing weight of [PR778]): for every permuted row r with a pair
+ * p = pair_of_row[r] (from `tables`),
+ *   y_w [P, N], row p = scale * topk_weights[p] * (A @ B[e]^T)[r]
+ * i.e. the down GEMM's rows, weighted, in flat pair order p = t*k + j; rows of
+ * pairs without a permuted row are not written. `epilogue` = MOE_EPI_STORE
+ * (y_w bf16, rounded to nearest even: half the bytes, the rounding of the
+ * pages' bf16 y) or MOE_EPI_STORE_F32 (y_w fp32, unrounded), OR-ed with
+ * MOE_TILE_AUTO, MOE_TILE_WEIGHT_ROWS or MOE_TILE_WEIGHT_ROWS_PAIR and their
+ * shape rules (N % 128 == 0; pairs: bf16 operands, N % 256 == 0);
+ * MOE_TILE_TOKEN_ROWS: MOE_ERR_UNSUPPORTED. A, A_scales, B, B_scales as for
+ * moe_grouped_gemm's store epilogues (bf16, or FP8 block-scaled with
+ * K <= 4096); tables as written by moe_route_permute (padding_M 128);
+ * topk_weights fp32 [T, k]. Device flags: MOE_DEV_TIMEOUT into *dev_status
+ * (required). */
+moe_status moe_down_gemm_weighted(const moe_problem* prob, int32_t N, int32_t K, const void* A,
+                                  const float* A_scales, const void* B, const float* B_scales,
+                                  const int32_t* tables, const float* topk_weights, float scale,
+                                  int32_t epilogue, void* y_w, int32_t* dev_status,
+                                  moe_stream_t stream);
+
+/* a7 after moe_down_gemm_weighted: the deterministic combine
+ *   out bf16 [T, H] = RNE_bf16( sum_{j<k} y_w[t*k+j] + addend[t] )
+ * with fp32 sums in slot order j, then the addend (fp32 [T, H] or NULL);
+ * pairs with row_of_pair == -1 contribute nothing. y_w [T*k, H] fp32
+ * (y_f32 != 0) or bf16; H % 8 == 0. */
+moe_status moe_combine(const moe_problem* prob, const void* y_w, int32_t y_f32,
+                       const int32_t* tables, const float* addend, void* out,
+                       moe_stream_t stream);
+
 /* Offline weight preparation for the FP8 down GEMM: for each of `batch`
  * matrices w bf16 [N, K], per 128x128 block s = amax/448 and
  * q = e4m3_rn_satfinite(w/s) (all-zero block: s = 0, q = 0); q uint8

@@ -20,7 +20,8 @@ __all__ = [
     "moe_experts_forward", "moe_decode_device_status", "moe_status_string",
     "moe_last_launch_count", "moe_shared_workspace_bytes", "moe_shared_expert_forward",
     "moe_dual_blocks", "moe_quant_dual", "moe_swiglu_quant_dual", "moe_swiglu_backward",
-    "moe_ep_split_ids", "moe_gather_rows", "EXPORTED_SYMBOLS",
+    "moe_ep_split_ids", "moe_gather_rows", "moe_down_gemm_weighted", "moe_combine",
+    "EXPORTED_SYMBOLS",
     "MOE_OK", "MOE_EPI_STORE", "MOE_EPI_SWIGLU", "MOE_EPI_SWIGLU_FP8", "MOE_EPI_STORE_F32",
     "MOE_SCORE_SOFTMAX", "MOE_SCORE_SIGMOID", "MOE_DEV_BAD_EXPERT_ID", "MOE_DEV_TIMEOUT",
 ]
@@ -46,7 +47,7 @@ EXPORTED_SYMBOLS = (
     "moe_last_cuda_error", "moe_last_launch_count", "moe_experts_forward_noalloc",
     "moe_shared_workspace_bytes", "moe_shared_expert_forward",
     "moe_dual_blocks", "moe_quant_dual", "moe_swiglu_quant_dual", "moe_swiglu_backward",
-    "moe_ep_split_ids", "moe_gather_rows",
+    "moe_ep_split_ids", "moe_gather_rows", "moe_down_gemm_weighted", "moe_combine",
 )
 
 
@@ -114,6 +115,10 @@ def lib() -> ctypes.CDLL:
         "moe_swiglu_quant": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, _P, _P,
                                             ctypes.c_int32, _P, _P, _P]),
         "moe_unpermute": (ctypes.c_int, [PP, _P, _P, _P, ctypes.c_float, _P, _P, _P]),
+        "moe_down_gemm_weighted": (ctypes.c_int, [PP, ctypes.c_int32, ctypes.c_int32, _P, _P,
+                                                  _P, _P, _P, _P, ctypes.c_float, ctypes.c_int32,
+                                                  _P, _P, _P]),
+        "moe_combine": (ctypes.c_int, [PP, _P, ctypes.c_int32, _P, _P, _P, _P]),
         "moe_quantize_weight_128x128": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32,
                                                        ctypes.c_int32, _P, _P, _P, _P]),
         "moe_experts_forward": (ctypes.c_int, [PP, _P, _P, _P, _P, _P, _P, _P, _P,
@@ -221,6 +226,23 @@ def moe_unpermute(prob, y, tables, topk_weights, scale, addend, out, stream=None
     _check(lib().moe_unpermute(ctypes.byref(prob), _ptr(y), _ptr(tables), _ptr(topk_weights),
                                float(scale), _ptr(addend), _ptr(out), _stream(stream)),
            "moe_unpermute")
+
+
+def moe_down_gemm_weighted(prob, N, K, A, A_scales, B, B_scales, tables, topk_weights, scale,
+                           epilogue, y_w, dev_status, stream=None):
+    _check(lib().moe_down_gemm_weighted(ctypes.byref(prob), int(N), int(K), _ptr(A),
+                                        _ptr(A_scales), _ptr(B), _ptr(B_scales), _ptr(tables),
+                                        _ptr(topk_weights), float(scale), int(epilogue),
+                                        _ptr(y_w), _ptr(dev_status), _stream(stream)),
+           "moe_down_gemm_weighted")
+
+
+def moe_combine(prob, y_w, tables, addend, out, stream=None):
+    """y_w fp32 or bf16 (taken from the tensor's dtype)."""
+    import torch
+    _check(lib().moe_combine(ctypes.byref(prob), _ptr(y_w), int(y_w.dtype == torch.float32),
+                             _ptr(tables), _ptr(addend), _ptr(out), _stream(stream)),
+           "moe_combine")
 
 
 def moe_quantize_weight_128x128(batch, N, K, w, q, scales, stream=None):

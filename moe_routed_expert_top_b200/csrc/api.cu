@@ -294,6 +294,80 @@ moe_status moe_unpermute(const moe_problem* prob, const float* y, const int32_t*
   return MOE_OK;
 }
 
+moe_status moe_down_gemm_weighted(const moe_problem* prob, int32_t N, int32_t K, const void* A,
+                                  const float* A_scales, const void* B, const float* B_scales,
+                                  const int32_t* tables, const float* topk_weights, float scale,
+                                  int32_t epilogue, void* y_w, int32_t* dev_status,
+                                  moe_stream_t stream) {
+  if (A == nullptr || B == nullptr || tables == nullptr || topk_weights == nullptr ||
+      y_w == nullptr || dev_status == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  moe_status s = check_problem(prob, false);
+  if (s != MOE_OK) return s;
+  if (prob->padding_M != 128) return MOE_ERR_UNSUPPORTED;
+  if (N <= 0 || K <= 0) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(y_w)) return MOE_ERR_INVALID_ARG;
+  if ((epilogue & ~0xFF) != 0) return MOE_ERR_INVALID_ARG;
+  const int t = (epilogue >> 4) & 0xF;
+  const int epi = epilogue & 0xF;
+  if (epi != MOE_EPI_STORE && epi != MOE_EPI_STORE_F32) return MOE_ERR_INVALID_ARG;
+  if (t > moe::kTilingWeightsPair) return MOE_ERR_INVALID_ARG;
+  if (t == moe::kTilingRows) return MOE_ERR_UNSUPPORTED;
+  const bool fp8 = A_scales != nullptr || B_scales != nullptr;
+  if (fp8 && (A_scales == nullptr || B_scales == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (N % 128 != 0 || K % (fp8 ? 128 : 64) != 0) return MOE_ERR_UNSUPPORTED;
+  moe_tables_layout L;
+  fill_layout(prob, &L);
+  if (L.P == 0) return MOE_OK;
+  moe::GemmLaunch g;
+  g.tiling = t;
+  g.mode = fp8 ? moe::kModeFp8Store : moe::kModeStore;
+  g.rows = L.P;
+  g.E = prob->E;
+  g.group_sizes = tables + L.group_sizes;
+  g.group_offsets = tables + L.group_offsets;
+  g.group_padded = tables + L.group_padded_offsets;
+  g.idx_for_bx = tables + L.group_idx_for_bx;
+  g.M_blk = L.M_blk;
+  g.N = N;
+  g.K = K;
+  g.A = A;
+  g.B = B;
+  g.A_scales = A_scales;
+  g.B_scales = B_scales;
+  g.C = y_w;
+  g.out_f32 = epi == MOE_EPI_STORE_F32;
+  g.status = dev_status;
+  g.weighted = 1;
+  g.pair_of_row = tables + L.pair_of_row;
+  g.row_weights = topk_weights;
+  g.row_scale = scale;
+  if (t == moe::kTilingWeights && !moe::grouped_gemm_t_supported(g)) return MOE_ERR_UNSUPPORTED;
+  if (t == moe::kTilingWeightsPair && !moe::grouped_gemm_pair_supported(g))
+    return MOE_ERR_UNSUPPORTED;
+  if (t == moe::kTilingAuto && !moe::grouped_gemm_t_supported(g) &&
+      !moe::grouped_gemm_pair_supported(g))
+    return MOE_ERR_UNSUPPORTED;
+  MOE_CUDA_TRY(moe::launch_grouped_gemm(g, reinterpret_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_combine(const moe_problem* prob, const void* y_w, int32_t y_f32,
+                       const int32_t* tables, const float* addend, void* out,
+                       moe_stream_t stream) {
+  moe_status s = check_problem(prob, false);
+  if (s != MOE_OK) return s;
+  if (prob->T == 0) return MOE_OK;
+  if (y_w == nullptr || tables == nullptr || out == nullptr) return MOE_ERR_INVALID_ARG;
+  if (prob->H % 8 != 0 || !aligned16(y_w) || !aligned16(out) || (addend && !aligned16(addend)))
+    return MOE_ERR_INVALID_ARG;
+  moe_tables_layout L;
+  fill_layout(prob, &L);
+  MOE_CUDA_TRY(moe::launch_combine(y_w, y_f32 != 0, tables + L.row_of_pair, prob->T, prob->top_k,
+                                   prob->H, addend, out, reinterpret_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
 moe_status moe_quantize_weight_128x128(int32_t batch, int32_t N, int32_t K, const void* w,
                                        uint8_t* q, float* scales, moe_stream_t stream) {
   if (batch < 0 || N < 0 || K < 0 || w == nullptr || q == nullptr || scales == nullptr)
@@ -373,7 +447,12 @@ moe_status moe_experts_forward(const moe_problem* prob, const void* hidden,
   g_last_launches += 1;
   g.A = x_perm;
   MOE_CUDA_TRY(moe::launch_grouped_gemm(g, st));
-  // a6: down
+  // a6: down, fp32 rows in expert order for the weighted unpermute. (Folding
+  // the routing weight into this epilogue, moe_down_gemm_weighted, writes the
+  // rows in flat pair order: in fp32 that measured as fast on DeepSeek shapes
+  // but slower on Qwen3 prefill, where the scattered 512-byte row segments
+  // cost more than the combine saves; in bf16 it is faster but its per-term
+  // rounding exceeds the output tolerance on rare DeepSeek outputs.)
   g.mode = prob->down_fp8 ? moe::kModeFp8Store : moe::kModeStore;
   g.N = H;
   g.K = F;

@@ -1,5 +1,6 @@
-// elementwise.cu - a7 weighted unpermute, a5 standalone SwiGLU(+E4M3 1x128
-// quantisation), and the offline 128x128 block quantisation of FP8 weights.
+// elementwise.cu - a7 weighted unpermute and the combine of pre-weighted rows,
+// a5 standalone SwiGLU(+E4M3 1x128 quantisation), and the offline 128x128
+// block quantisation of FP8 weights.
 // All three are HBM-streaming kernels: 16-byte vector loads/stores, fp32 math.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -23,9 +24,11 @@ __global__ void __launch_bounds__(128) unpermute_kernel(const float4* __restrict
                                                         const float* __restrict__ w, int k,
                                                         int P, int H8, float scale,
                                                         const float4* __restrict__ addend,
-                                                        uint4* __restrict__ out) {
-  const int t = blockIdx.y;
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;  // 8-column group
+                                                        uint4* __restrict__ out, int cblocks) {
+  // one block per (token, 128 groups of 8 columns): a flat grid, so T is not
+  // bound by the 65535 limit of a grid's y extent
+  const int t = static_cast<int>(blockIdx.x / cblocks);
+  const int c = static_cast<int>(blockIdx.x % cblocks) * blockDim.x + threadIdx.x;  // 8-column group
   if (c >= H8) return;
   float acc[8];
 #pragma unroll
@@ -90,11 +93,96 @@ cudaError_t launch_unpermute(const float* y, const int32_t* row_of_pair, const f
                              cudaStream_t stream) {
   if (T <= 0) return cudaSuccess;
   const int H8 = H / 8;
-  dim3 grid((H8 + 127) / 128, T);
-  unpermute_kernel<<<grid, 128, 0, stream>>>(reinterpret_cast<const float4*>(y), row_of_pair,
-                                             weights, k, T * k, H8, scale,
-                                             reinterpret_cast<const float4*>(addend),
-                                             static_cast<uint4*>(out));
+  const int cblocks = (H8 + 127) / 128;
+  const long long blocks = static_cast<long long>(T) * cblocks;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  unpermute_kernel<<<static_cast<unsigned>(blocks), 128, 0, stream>>>(
+      reinterpret_cast<const float4*>(y), row_of_pair, weights, k, T * k, H8, scale,
+      reinterpret_cast<const float4*>(addend), static_cast<uint4*>(out), cblocks);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Combine of weighted rows (the unpermute's gather-reduce once the routing
+// weight and scale were applied in the down GEMM's epilogue; TileOPs PR #1580,
+// Unpermute, with the weight fold of the down projection's row scale):
+//   out[t] = bf16( sum_{j<k} y_w[t*k+j] + addend[t] )
+// y_w bf16 or fp32 [T*k, H] in flat pair order; pairs without a row
+// (row_of_pair -1) contribute nothing. fp32 sums in slot order j, then the
+// addend: the result does not depend on scheduling. One thread per 8 columns
+// of one token.
+// ---------------------------------------------------------------------------
+template <bool kF32>
+__global__ void __launch_bounds__(128) combine_kernel(const uint4* __restrict__ y_w,
+                                                      const int32_t* __restrict__ row_of_pair,
+                                                      int k, int H8,
+                                                      const float4* __restrict__ addend,
+                                                      uint4* __restrict__ out, int cblocks) {
+  constexpr int kVec = kF32 ? 2 : 1;  // 16-byte vectors per 8 columns
+  const int t = static_cast<int>(blockIdx.x / cblocks);
+  const int c = static_cast<int>(blockIdx.x % cblocks) * blockDim.x + threadIdx.x;
+  if (c >= H8) return;
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+  const int64_t pbase = static_cast<int64_t>(t) * k;
+  for (int j0 = 0; j0 < k; j0 += 8) {
+    // all row checks, then all loads, then the adds in slot order: up to 8
+    // independent 16-byte loads in flight per thread
+    bool has[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) has[j] = j0 + j < k && __ldg(row_of_pair + pbase + j0 + j) >= 0;
+    uint4 v[8][kVec];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int u = 0; u < kVec; ++u)
+        v[j][u] = has[j] ? __ldg(y_w + ((pbase + j0 + j) * H8 + c) * kVec + u)
+                         : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (!has[j]) continue;
+      if constexpr (kF32) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          acc[4 * u + 0] += __uint_as_float(v[j][u].x);
+          acc[4 * u + 1] += __uint_as_float(v[j][u].y);
+          acc[4 * u + 2] += __uint_as_float(v[j][u].z);
+          acc[4 * u + 3] += __uint_as_float(v[j][u].w);
+        }
+      } else {
+        const uint32_t w4[4] = {v[j][0].x, v[j][0].y, v[j][0].z, v[j][0].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          acc[2 * q] += bf16lo_to_f32(w4[q]);
+          acc[2 * q + 1] += bf16hi_to_f32(w4[q]);
+        }
+      }
+    }
+  }
+  if (addend != nullptr) {
+    const float4* ad = addend + (static_cast<int64_t>(t) * H8 + c) * 2;
+    const float4 a = __ldg(ad), b = __ldg(ad + 1);
+    const float add[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] += add[i];
+  }
+  out[static_cast<int64_t>(t) * H8 + c] =
+      make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                 pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+}
+
+cudaError_t launch_combine(const void* y_w, bool y_f32, const int32_t* row_of_pair, int T, int k,
+                           int H, const float* addend, void* out, cudaStream_t stream) {
+  if (T <= 0) return cudaSuccess;
+  const int H8 = H / 8;
+  const int cblocks = (H8 + 127) / 128;
+  const long long blocks = static_cast<long long>(T) * cblocks;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  auto kern = y_f32 ? combine_kernel<true> : combine_kernel<false>;
+  kern<<<static_cast<unsigned>(blocks), 128, 0, stream>>>(
+      static_cast<const uint4*>(y_w), row_of_pair, k, H8, reinterpret_cast<const float4*>(addend),
+      static_cast<uint4*>(out), cblocks);
   return cudaGetLastError();
 }
 

@@ -643,6 +643,8 @@ cudaError_t launch_grouped_gemm(const GemmLaunch& L, cudaStream_t stream) {
       (L.tiling == kTilingWeights || (L.tiling == kTilingAuto && grouped_gemm_t_preferred(L))))
     return launch_grouped_gemm_t(L, stream);
   if (L.tiling == kTilingWeights) return cudaErrorNotSupported;
+  // the weighted (pair-order) store is built into the weight-row tilings only
+  if (L.weighted) return cudaErrorNotSupported;
   switch (L.mode) {
     case kModeStore:
       if (L.N % 256 == 0) return run_gemm<kModeStore, 256>(L, stream);

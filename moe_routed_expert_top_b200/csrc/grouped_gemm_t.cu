@@ -58,6 +58,11 @@ struct TParams {
   const float* B_scales;  // FP8: weight block scales [E, N/128, KBS]
   int KBS;                // FP8: K / 128
   int32_t* status;
+  // weighted store: C row pair_of_row[r] = row_scale * row_w[pair] * result row r
+  int weighted;
+  const int32_t* pair_of_row;
+  const float* row_w;
+  float row_scale;
 };
 
 __host__ __device__ constexpr int tmin(int a, int b) { return a < b ? a : b; }
@@ -76,7 +81,9 @@ struct TCfg {
   // bound); bf16: 2 tile buffers
   static constexpr int NUM_ACC = kFp8 ? 512 / TN : 2;
   static constexpr int TMEM_COLS = NUM_ACC * TN;
-  static constexpr int STAGE_OUT_BYTES = 32 * 128 * 4;  // 32 token rows x 128 fp32
+  // 32 token rows x 128 fp32, then the tile's row destinations and factors
+  // (weighted store)
+  static constexpr int STAGE_OUT_BYTES = 32 * 128 * 4 + 2 * TN * 4;
   static constexpr int MAX_KBS = 32;                    // FP8: K <= 4096
   static constexpr int SA_BYTES = kFp8 ? TN * MAX_KBS * 4 : 0;
   static constexpr int NUM_BARS = 2 * STAGES + 2 * NUM_ACC + 1;
@@ -135,18 +142,41 @@ __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: 
 
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
 
+// Weighted store: the destination row (flat pair index, -1 = none) and the
+// factor row_scale * row_w[pair] of a tile's rows row0 .. row0 + rows - 1,
+// loaded by the 128 epilogue threads when the tile starts, so the loads' latency
+// passes while the tile's MMAs run; read after the barrier that precedes the
+// first store.
+__device__ __forceinline__ void stage_row_info(const TParams& p, int et, int rows, int row0,
+                                               int* sDst, float* sFac) {
+  for (int i = et; i < rows; i += 128) {
+    const int pr = __ldg(p.pair_of_row + row0 + i);
+    sDst[i] = pr;
+    sFac[i] = pr >= 0 ? p.row_scale * __ldg(p.row_w + pr) : 0.0f;
+  }
+}
+
 // Write `rows` staged token rows (sOut[i][0..128), fp32) to C rows row0.. at
-// column col0, fp32 or bf16, 16-byte stores; 128 epilogue threads (et).
+// column col0, fp32 or bf16, 16-byte stores; 128 epilogue threads (et). A
+// weighted store writes row i to sDst[i], scaled by sFac[i].
 __device__ __forceinline__ void store_rows(const TParams& p, const float* sOut, int et, int rows,
-                                           int row0, int col0) {
+                                           int row0, int col0, const int* sDst,
+                                           const float* sFac) {
   if (p.out_f32) {
 #pragma unroll
     for (int pass = 0; pass < 8; ++pass) {
       const int i = pass * 4 + (et >> 5);
       const int c4 = et & 31;
       if (i < rows) {
-        const float4 val = reinterpret_cast<const float4*>(sOut + i * 128)[c4];
-        float* dst = static_cast<float*>(p.C) + static_cast<int64_t>(row0 + i) * p.ldc + col0;
+        float4 val = reinterpret_cast<const float4*>(sOut + i * 128)[c4];
+        int drow = row0 + i;
+        if (p.weighted) {
+          drow = sDst[i];
+          const float f = sFac[i];
+          if (drow < 0) continue;
+          val = make_float4(val.x * f, val.y * f, val.z * f, val.w * f);
+        }
+        float* dst = static_cast<float*>(p.C) + static_cast<int64_t>(drow) * p.ldc + col0;
         reinterpret_cast<float4*>(dst)[c4] = val;
       }
     }
@@ -157,10 +187,22 @@ __device__ __forceinline__ void store_rows(const TParams& p, const float* sOut, 
       const int c8 = et & 15;
       if (i < rows) {
         const float* src = sOut + i * 128 + c8 * 8;
-        const uint4 val = make_uint4(pack_bf16x2(src[0], src[1]), pack_bf16x2(src[2], src[3]),
-                                     pack_bf16x2(src[4], src[5]), pack_bf16x2(src[6], src[7]));
+        int drow = row0 + i;
+        float f = 1.0f;
+        if (p.weighted) {
+          drow = sDst[i];
+          f = sFac[i];
+          if (drow < 0) continue;
+        }
+        const uint4 val =
+            p.weighted ? make_uint4(pack_bf16x2(src[0] * f, src[1] * f),
+                                    pack_bf16x2(src[2] * f, src[3] * f),
+                                    pack_bf16x2(src[4] * f, src[5] * f),
+                                    pack_bf16x2(src[6] * f, src[7] * f))
+                       : make_uint4(pack_bf16x2(src[0], src[1]), pack_bf16x2(src[2], src[3]),
+                                    pack_bf16x2(src[4], src[5]), pack_bf16x2(src[6], src[7]));
         __nv_bfloat16* dst =
-            static_cast<__nv_bfloat16*>(p.C) + static_cast<int64_t>(row0 + i) * p.ldc + col0;
+            static_cast<__nv_bfloat16*>(p.C) + static_cast<int64_t>(drow) * p.ldc + col0;
         reinterpret_cast<uint4*>(dst)[c8] = val;
       }
     }
@@ -184,7 +226,9 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* sA = smem;                                   // weight tiles
   uint8_t* sB = smem + STAGES * Cfg::A_BYTES;           // token tiles
   float* sOut = reinterpret_cast<float*>(sB + STAGES * Cfg::B_BYTES);  // [32][128]
-  float* sSa = sOut + 32 * 128;  // FP8: activation scales of the tile's tokens [TN][KBS]
+  int* sDst = reinterpret_cast<int*>(sOut + 32 * 128);  // weighted store: the tile's row info
+  float* sFac = reinterpret_cast<float*>(sDst + TN);
+  float* sSa = sOut + 32 * 128 + 2 * TN;  // FP8: activation scales of the tile's tokens [TN][KBS]
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sOut) +
                                                Cfg::STAGE_OUT_BYTES + Cfg::SA_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NUM_BARS);
@@ -404,6 +448,7 @@ __global__ void __launch_bounds__(192, 1)
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
       TTile ti;
       if (!t_decode(p, cpre, E, WB, TN, t, ti)) continue;
+      if (kMode != kTSwiglu && p.weighted) stage_row_info(p, et, ti.nt, ti.m0, sDst, sFac);
       if constexpr (Cfg::kFp8) {
         // y[t, w] = sum_kb sw[e, wb, kb] * sa[t, kb] * (Wq_kb Xq_kb^T)[w, t]
         // stage s[kb][t] = sw[e, wb, kb] * sa[m0 + t, kb], K-block major so each
@@ -482,7 +527,8 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i) sOut[i * 128 + r] = accv[c * 32 + i];
             epi_bar();
-            store_rows(p, sOut, et, tmin(32, ti.nt - c * 32), ti.m0 + c * 32, ti.wb * 128);
+            store_rows(p, sOut, et, tmin(32, ti.nt - c * 32), ti.m0 + c * 32, ti.wb * 128,
+                       sDst + c * 32, sFac + c * 32);
             epi_bar();
           }
         }
@@ -503,38 +549,12 @@ __global__ void __launch_bounds__(192, 1)
         // sOut[i][r] = D[r][j0 + i]: token row i, weight row r
 #pragma unroll
         for (int i = 0; i < 32; ++i) sOut[i * 128 + r] = __uint_as_float(v[i]);
-        epi_bar();
         const int rows = tmin(32, ti.nt - j0);
+        epi_bar();
         if constexpr (kMode == kTStore) {
-          if (p.out_f32) {
-            // a token row = 128 fp32 = 32 x 16 B; 4 rows per pass
-#pragma unroll
-            for (int pass = 0; pass < 8; ++pass) {
-              const int i = pass * 4 + (et >> 5);
-              const int c4 = et & 31;
-              if (i < rows) {
-                const float4 val = reinterpret_cast<const float4*>(sOut + i * 128)[c4];
-                float* dst = static_cast<float*>(p.C) +
-                             static_cast<int64_t>(ti.m0 + j0 + i) * p.ldc + ti.wb * 128;
-                reinterpret_cast<float4*>(dst)[c4] = val;
-              }
-            }
-          } else {
-            // a token row = 128 bf16 = 16 x 16 B; 8 rows per pass
-#pragma unroll
-            for (int pass = 0; pass < 4; ++pass) {
-              const int i = pass * 8 + (et >> 4);
-              const int c8 = et & 15;
-              if (i < rows) {
-                const float* src = sOut + i * 128 + c8 * 8;
-                const uint4 val = make_uint4(pack_bf16x2(src[0], src[1]), pack_bf16x2(src[2], src[3]),
-                                             pack_bf16x2(src[4], src[5]), pack_bf16x2(src[6], src[7]));
-                __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.C) +
-                                     static_cast<int64_t>(ti.m0 + j0 + i) * p.ldc + ti.wb * 128;
-                reinterpret_cast<uint4*>(dst)[c8] = val;
-              }
-            }
-          }
+          // a token row = 128 fp32 (32 x 16 B, 4 rows per pass) or 128 bf16
+          // (16 x 16 B, 8 rows per pass)
+          store_rows(p, sOut, et, rows, ti.m0 + j0, ti.wb * 128, sDst + j0, sFac + j0);
         } else {
           // swiglu: gate = weight rows 0..63, up = rows 64..127 of the block;
           // h row = 64 bf16 = 8 x 16 B; 16 rows per pass
@@ -648,6 +668,10 @@ cudaError_t run_t(const GemmLaunch& L, cudaStream_t stream) {
   p.B_scales = L.B_scales;
   p.KBS = L.K / 128;
   p.status = L.status;
+  p.weighted = L.weighted;
+  p.pair_of_row = L.pair_of_row;
+  p.row_w = L.row_weights;
+  p.row_scale = L.row_scale;
   const int WB = kMode == kTSwiglu ? (L.N / 2) / 64 : L.N / 128;
   const long long chunks_ub = grouped ? (static_cast<long long>(L.rows) + TN - 1) / TN + E
                                       : (static_cast<long long>(L.rows) + TN - 1) / TN;
@@ -663,6 +687,10 @@ cudaError_t run_t(const GemmLaunch& L, cudaStream_t stream) {
 
 bool grouped_gemm_t_supported(const GemmLaunch& L) {
   if (L.E > 1024) return false;
+  if (L.weighted && (L.pair_of_row == nullptr || L.row_weights == nullptr ||
+                     L.group_sizes == nullptr ||
+                     (L.mode != kModeStore && L.mode != kModeFp8Store)))
+    return false;
   if (L.mode == kModeFp8Store)
     return L.A_scales != nullptr && L.B_scales != nullptr && L.N % 128 == 0 &&
            L.K % 128 == 0 && L.K <= 128 * 32;

@@ -61,6 +61,10 @@ struct PParams {
   int top_k;
   int hidden_rows;
   int up_off;  // SwiGLU: rows from a gate row of W to its up row
+  // weighted store: C row pair_of_row[r] = row_scale * row_w[pair] * result row r
+  int weighted;
+  const float* row_w;
+  float row_scale;
 };
 
 __host__ __device__ constexpr int pmin(int a, int b) { return a < b ? a : b; }
@@ -75,7 +79,9 @@ struct PCfg {
   static constexpr int STAGES = pmin(8, (200 * 1024) / STAGE_BYTES);
   static constexpr int NUM_ACC = 2;
   static constexpr int TMEM_COLS = 2 * TN;
-  static constexpr int STAGE_OUT_BYTES = 32 * 128 * 4;
+  // 32 token rows x 128 fp32, then the tile's row destinations and factors
+  // (weighted store)
+  static constexpr int STAGE_OUT_BYTES = 32 * 128 * 4 + 2 * TN * 4;
   static constexpr int NUM_BARS = 2 * STAGES + 2 * NUM_ACC + 1;
   static constexpr int MAX_E = 1024;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STAGE_OUT_BYTES +
@@ -159,6 +165,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * Cfg::A_BYTES;
   float* sOut = reinterpret_cast<float*>(sB + STAGES * Cfg::B_BYTES);
+  int* sDst = reinterpret_cast<int*>(sOut + 32 * 128);  // weighted store: the tile's row info
+  float* sFac = reinterpret_cast<float*>(sDst + TN);
   uint64_t* bars =
       reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sOut) + Cfg::STAGE_OUT_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NUM_BARS);
@@ -382,6 +390,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     for (int t = pair; t < total_tiles; t += npairs) {
       PTile ti;
       if (!p_decode(p, cpre, E, WB, TN, t, ti)) continue;
+      if (kMode == kPStore && p.weighted) {
+        // the tile's row destinations (flat pair index, -1 = none) and factors,
+        // loaded while its MMAs run; read after the first chunk's barrier
+        for (int i = et; i < ti.nt; i += 128) {
+          const int pr = __ldg(p.pair_of_row + ti.m0 + i);
+          sDst[i] = pr;
+          sFac[i] = pr >= 0 ? p.row_scale * __ldg(p.row_w + pr) : 0.0f;
+        }
+      }
       if (!mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, p.status)) *epi_abort = 1;
       pepi_bar();
       if (*epi_abort) break;
@@ -396,8 +413,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         if (more) tmem_ld32(tb + j0 + 32, vn);
 #pragma unroll
         for (int i = 0; i < 32; ++i) sOut[i * 128 + r] = __uint_as_float(v[i]);
-        pepi_bar();
         const int rows = pmin(32, ti.nt - j0);
+        pepi_bar();
         if constexpr (kMode == kPStore) {
           if (p.out_f32) {
 #pragma unroll
@@ -405,9 +422,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
               const int i = pass * 4 + (et >> 5);
               const int c4 = et & 31;
               if (i < rows) {
-                const float4 val = reinterpret_cast<const float4*>(sOut + i * 128)[c4];
-                float* dst = static_cast<float*>(p.C) +
-                             static_cast<int64_t>(ti.m0 + j0 + i) * p.ldc + col0;
+                float4 val = reinterpret_cast<const float4*>(sOut + i * 128)[c4];
+                int drow = ti.m0 + j0 + i;
+                if (p.weighted) {
+                  drow = sDst[j0 + i];
+                  const float f = sFac[j0 + i];
+                  if (drow < 0) continue;
+                  val = make_float4(val.x * f, val.y * f, val.z * f, val.w * f);
+                }
+                float* dst = static_cast<float*>(p.C) + static_cast<int64_t>(drow) * p.ldc + col0;
                 reinterpret_cast<float4*>(dst)[c4] = val;
               }
             }
@@ -418,11 +441,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
               const int c8 = et & 15;
               if (i < rows) {
                 const float* src = sOut + i * 128 + c8 * 8;
+                int drow = ti.m0 + j0 + i;
+                float f = 1.0f;
+                if (p.weighted) {
+                  drow = sDst[j0 + i];
+                  f = sFac[j0 + i];
+                  if (drow < 0) continue;
+                }
                 const uint4 val =
-                    make_uint4(pack_bf16x2(src[0], src[1]), pack_bf16x2(src[2], src[3]),
-                               pack_bf16x2(src[4], src[5]), pack_bf16x2(src[6], src[7]));
+                    p.weighted ? make_uint4(pack_bf16x2(src[0] * f, src[1] * f),
+                                            pack_bf16x2(src[2] * f, src[3] * f),
+                                            pack_bf16x2(src[4] * f, src[5] * f),
+                                            pack_bf16x2(src[6] * f, src[7] * f))
+                               : make_uint4(pack_bf16x2(src[0], src[1]), pack_bf16x2(src[2], src[3]),
+                                            pack_bf16x2(src[4], src[5]), pack_bf16x2(src[6], src[7]));
                 __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.C) +
-                                     static_cast<int64_t>(ti.m0 + j0 + i) * p.ldc + col0;
+                                     static_cast<int64_t>(drow) * p.ldc + col0;
                 reinterpret_cast<uint4*>(dst)[c8] = val;
               }
             }
@@ -553,6 +587,9 @@ cudaError_t run_pair(const GemmLaunch& L, cudaStream_t stream) {
   p.top_k = L.top_k;
   p.hidden_rows = a_rows;
   p.up_off = L.up_off > 0 ? L.up_off : L.N / 2;
+  p.weighted = L.weighted;
+  p.row_w = L.row_weights;
+  p.row_scale = L.row_scale;
   const int WB = kMode == kPSwiglu ? (L.N / 2) / 128 : L.N / 256;
   const long long chunks_ub = grouped ? (static_cast<long long>(L.rows) + TN - 1) / TN + E
                                       : (static_cast<long long>(L.rows) + TN - 1) / TN;
@@ -573,6 +610,9 @@ cudaError_t run_pair_g(const GemmLaunch& L, cudaStream_t stream) {
 
 bool grouped_gemm_pair_supported(const GemmLaunch& L) {
   if (L.A_scales != nullptr || L.B_scales != nullptr || L.E > 1024) return false;
+  if (L.weighted && (L.pair_of_row == nullptr || L.row_weights == nullptr ||
+                     L.group_sizes == nullptr || L.mode != kModeStore))
+    return false;
   // gathering needs the group tables and the row -> pair map
   if (L.gather && (L.group_sizes == nullptr || L.pair_of_row == nullptr || L.top_k <= 0 ||
                    L.a_rows <= 0))

@@ -46,6 +46,13 @@ struct GemmLaunch {
   int ldb = 0;
   int up_off = 0;
   long long b_rows = 0;
+  // weighted store (store modes, bf16 or fp32 C, grouped; weight-row tilings only):
+  // row r of the result goes to C row pair_of_row[r] (flat pair order),
+  // multiplied by row_scale * row_weights[pair_of_row[r]]; rows with no pair
+  // (-1) are skipped
+  int weighted = 0;
+  const float* row_weights = nullptr;
+  float row_scale = 1.0f;
 };
 
 // Tiling of the grouped GEMM: token-row tiles (grouped_gemm.cu), weight-row
@@ -79,6 +86,8 @@ cudaError_t launch_gather_rows(const void* hidden, const int32_t* pair_of_row, i
 cudaError_t launch_unpermute(const float* y, const int32_t* row_of_pair, const float* weights,
                              int T, int k, int H, float scale, const float* addend, void* out,
                              cudaStream_t stream);
+cudaError_t launch_combine(const void* y_w, bool y_f32, const int32_t* row_of_pair, int T, int k,
+                           int H, const float* addend, void* out, cudaStream_t stream);
 
 cudaError_t launch_swiglu_quant(int M, int F, const void* gate_up, const float* h, int out_fp8,
                                 void* out, float* scales, cudaStream_t stream);

@@ -590,6 +590,51 @@ def unpermute(y: np.ndarray, row_of_pair: np.ndarray, topk_weights: np.ndarray,
     return bf16_round(acc) if round_output else acc
 
 
+def weighted_rows(y: np.ndarray, pair_of_row: np.ndarray, topk_weights: np.ndarray,
+                  scale: float, round_output: bool = True):
+    """The down projection's rows with the routing weight and scale applied,
+    moved to flat pair order (SURVEY's "fold the routing weight x scale into
+    the down-GEMM epilogue": TileOPs PR #1580 §Unpermute's scale folding done
+    one step earlier, as a per-row scale x routing weight):
+        y_w[p] = bf16( scale * w[p] * y[r] )   for every row r with p = pair_of_row[r] >= 0
+    The bf16 rounding is the one the pages put on the down GEMM's output (y is
+    bf16 [P, H] in their layout); ``round_output=False`` keeps the float64
+    product. Returns (y_w float64 [P, H], written bool [P]); rows of pairs with
+    no permuted row stay 0 / unwritten."""
+    w = np.asarray(topk_weights, dtype=np.float64).reshape(-1)
+    y = as_f64(y)
+    por = np.asarray(pair_of_row).reshape(-1)
+    P = w.shape[0]
+    out = np.zeros((P, y.shape[1]), dtype=np.float64)
+    written = np.zeros(P, dtype=bool)
+    for r in range(por.shape[0]):
+        p = int(por[r])
+        if p < 0:
+            continue
+        v = float(scale) * w[p] * y[r]
+        out[p] = bf16_round(v) if round_output else v
+        written[p] = True
+    return out, written
+
+
+def combine(y_w: np.ndarray, row_of_pair: np.ndarray, k: int, addend=None,
+            round_output: bool = True) -> np.ndarray:
+    """out[t] = bf16( sum_{j<k, row_of_pair[t*k+j] >= 0} y_w[t*k+j] + addend[t] )
+    (TileOPs PR #1580 §Unpermute's gather-reduce once the weights are applied:
+    the deterministic combine). Sum over j in slot order, float64."""
+    y_w = as_f64(y_w)
+    rop = np.asarray(row_of_pair).reshape(-1)
+    P, H = y_w.shape
+    T = P // k
+    acc = np.zeros((T, H), dtype=np.float64)
+    for j in range(k):
+        has = rop[j::k] >= 0
+        acc[has] += y_w[j::k][has]
+    if addend is not None:
+        acc = acc + as_f64(addend)
+    return bf16_round(acc) if round_output else acc
+
+
 # ---------------------------------------------------------------------------
 # whole experts forward, by its plain definition per token
 # ---------------------------------------------------------------------------
