@@ -529,7 +529,106 @@ OPS = {
     "swiglu_backward_32k": dict(kind="backward", M=32768, K=2048),
     "swiglu_backward_128k": dict(kind="backward", M=131072, K=4096),
 }
+# the down GEMM with the routing weight folded into its epilogue, then the
+# combine, on a whole workload (rows stored bf16 or fp32)
+for _w in ("qwen3_decode", "qwen3_prefill", "dsv3_prefill", "dsv3_decode_fp8"):
+    for _d in ("bf16", "f32"):
+        OPS[f"fold_{_w}_{_d}"] = dict(kind="fold", workload=_w, rows=_d)
 OP_METRIC = "training-FP8 op ms + achieved GB/s, % of B200 HBM roofline (1 GPU)"
+FOLD_METRIC = ("down GEMM with the routing weight folded in + combine, ms per layer, "
+               "% of B200 roofline (1 GPU)")
+
+
+def run_fold(args, device, spec) -> dict:
+    """Weighted down GEMM + combine on a workload, timed beside the forward's
+    own down GEMM (fp32 rows in expert order) + weighted unpermute."""
+    import moe_routed_expert_top_b200 as M
+    cfg = get_config(spec["workload"])
+    M, layer, hidden, ids, weights, _ = build_layer(cfg, device)
+    peaks = load_peaks()
+    wm = work_model(cfg, ids.cpu().numpy())
+    prob = layer.problem(cfg.T)
+    L = M.moe_get_tables_layout(prob)
+    P, H, F, T = L["P"], cfg.H, cfg.F, cfg.T
+    tables = torch.empty(L["total_int32"], dtype=torch.int32, device=device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    x_perm = torch.empty(P, H, dtype=torch.bfloat16, device=device)
+    M.moe_route_permute(prob, None, ids, None, hidden, x_perm, tables, status)
+    if cfg.down_fp8:
+        h = torch.empty(P, F, dtype=torch.uint8, device=device)
+        hs = torch.empty(P, F // 128, dtype=torch.float32, device=device)
+    else:
+        h = torch.empty(P, F, dtype=torch.bfloat16, device=device)
+        hs = None
+    M.moe_grouped_gemm(prob, 0, 2 * F, H, x_perm, None, layer.w_gate_up, None, tables,
+                       M.MOE_EPI_SWIGLU_FP8 if cfg.down_fp8 else M.MOE_EPI_SWIGLU, h, hs, None,
+                       status)
+    del x_perm
+    f32 = spec["rows"] == "f32"
+    y_w = torch.empty(P, H, dtype=torch.float32 if f32 else torch.bfloat16, device=device)
+    y = torch.empty(P, H, dtype=torch.float32, device=device)
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=device)
+    s = cfg.routed_scaling_factor
+    down_w = lambda: M.moe_down_gemm_weighted(prob, H, F, h, hs, layer.w_down,
+                                              layer.w_down_scales, tables, weights, s,
+                                              M.MOE_EPI_STORE_F32 if f32 else M.MOE_EPI_STORE,
+                                              y_w, status)
+    comb = lambda: M.moe_combine(prob, y_w, tables, None, out)
+    down = lambda: M.moe_grouped_gemm(prob, 0, H, F, h, hs, layer.w_down, layer.w_down_scales,
+                                      tables, M.MOE_EPI_STORE_F32, y, None, None, status)
+    unp = lambda: M.moe_unpermute(prob, y, tables, weights, s, None, out)
+
+    def fold():
+        down_w()
+        comb()
+
+    def plain():
+        down()
+        unp()
+
+    fns = {"fold": fold, "down_weighted": down_w, "combine": comb, "forward_path": plain,
+           "down_f32": down, "unpermute": unp}
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    for fn in fns.values():
+        for _ in range(args.warmup):
+            fn()
+    torch.cuda.synchronize()
+    res = {}
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for name, fn in fns.items():
+            res[name] = statistics.median(time_steps(fn, args.steps, flush, stream))
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, "device status flag set"
+    # the weighted down GEMM: its weights, its A rows (h), its pair-order rows
+    rb = 4 if f32 else 2
+    dn_bytes = wm["down_bytes"] - P * H * 4 + P * H * rb
+    t_s = res["down_weighted"] * 1e-3
+    t_byte = dn_bytes / (peaks["hbm_gbs"] * 1e9)
+    # FP8 operands: the measured bf16 peak x the nominal fp8/bf16 ratio of 2
+    mma_peak = peaks["bf16_tflops"] * (2.0 if cfg.down_fp8 else 1.0)
+    t_flop = wm["down_flops"] / (mma_peak * 1e12)
+    tensor = t_flop > t_byte
+    achieved = (wm["down_flops"] / t_s / 1e12) if tensor else (dn_bytes / t_s / 1e9)
+    peak = mma_peak if tensor else peaks["hbm_gbs"]
+    return {
+        "metric": FOLD_METRIC, "op": args.op, "value": round(res["fold"], 4), "unit": "ms",
+        "higher_is_better": False, "steps": args.steps, "warmup": args.warmup,
+        "dtype": ("e4m3 x e4m3 (block-scaled)" if cfg.down_fp8 else "bf16") +
+                 (", fp32 rows" if f32 else ", bf16 rows"),
+        "data": "synthetic", "config": {"workload": cfg.name, "rows": spec["rows"], "T": T,
+                                        "E": cfg.E, "top_k": cfg.top_k, "H": H, "F": F,
+                                        "l2": "flushed (512 MiB write) before each call"},
+        "stages_ms": {k: round(v, 4) for k, v in res.items()},
+        "roofline": {"bound": "tensor" if tensor else "hbm", "kernel": "down_weighted",
+                     "achieved": round(achieved, 1), "peak": peak,
+                     "unit": "TFLOP/s" if tensor else "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": None, "algorithmic_bytes": int(dn_bytes),
+                     "flops": wm["down_flops"]},
+        "timing": "median of per-call CUDA events on the launching stream; forward_path = "
+                  "the forward's own down GEMM (fp32 rows, expert order) + unpermute",
+        "clocks": clk.summary(),
+    }
 
 
 def run_op(args, device) -> dict:
@@ -537,6 +636,8 @@ def run_op(args, device) -> dict:
     from moe_routed_expert_top_b200 import build
     build.build()
     spec = dict(OPS[args.op])
+    if spec["kind"] == "fold":
+        return run_fold(args, device, spec)
     if args.override:       # e.g. M=32768: a smaller case of the same op (profiling)
         for item in args.override.split(","):
             key, val = item.split("=", 1)

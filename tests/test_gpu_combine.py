@@ -303,3 +303,54 @@ def test_weighted_down_needs_a_weight_row_tiling():
     ref = O.experts_forward(gu.f64(hidden), ids_np, w_np, gu.f64(wts["w_gate_up"]),
                             gu.f64(wts["w_down"]), cfg.routed_scaling_factor)
     gu.assert_within_tol(gu.f64(out), ref, "forward H=192")
+
+
+@pytest.mark.parametrize("name,f32", [("qwen3_prefill", True), ("qwen3_prefill", False),
+                                      ("dsv3_decode_fp8", True)])
+def test_weighted_chain_full_size_sampled(name, f32):
+    """Full-size workloads: tables, gate+up (SwiGLU, or SwiGLU + FP8 1x128),
+    the weighted down GEMM (bf16 or FP8 block-scaled) and the combine, against
+    the oracle's forward on seeded token samples (including the tokens of the
+    most and the least loaded experts)."""
+    gu = _gu()
+    import moe_routed_expert_top_b200 as M
+    from moe_routed_expert_top_b200.layer import RoutedExperts
+    from tests.test_gpu_forward import _inputs, _oracle
+    cfg = get_config(name)
+    hidden, ids, w, weights = _inputs(cfg)
+    layer = RoutedExperts(weights["w_gate_up"], weights["w_down"], cfg.top_k, cfg.score_fn,
+                          cfg.renormalize, cfg.routed_scaling_factor, cfg.down_fp8)
+    prob = layer.problem(cfg.T)
+    L, tables, status, x_perm = gu.gpu_tables(cfg, ids, hidden=hidden)
+    P, H, F = L["P"], cfg.H, cfg.F
+    if cfg.down_fp8:
+        h = torch.empty(P, F, dtype=torch.uint8, device="cuda")
+        hs = torch.empty(P, F // 128, dtype=torch.float32, device="cuda")
+        epi = M.MOE_EPI_SWIGLU_FP8
+    else:
+        h = torch.empty(P, F, dtype=torch.bfloat16, device="cuda")
+        hs, epi = None, M.MOE_EPI_SWIGLU
+    M.moe_grouped_gemm(prob, 0, 2 * F, H, x_perm, None, layer.w_gate_up, None, tables, epi, h,
+                       hs, None, status)
+    y_w = torch.full((P, H), float("nan"), dtype=torch.float32 if f32 else torch.bfloat16,
+                     device="cuda")
+    M.moe_down_gemm_weighted(prob, H, F, h, hs, layer.w_down, layer.w_down_scales, tables,
+                             torch.from_numpy(w).cuda(), cfg.routed_scaling_factor,
+                             M.MOE_EPI_STORE_F32 if f32 else M.MOE_EPI_STORE, y_w, status)
+    out = torch.empty(cfg.T, H, dtype=torch.bfloat16, device="cuda")
+    M.moe_combine(prob, y_w, tables, None, out)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert torch.isfinite(y_w.float()).all()          # every pair row written
+    rng = np.random.default_rng(8)
+    sizes = np.bincount(ids.reshape(-1), minlength=cfg.E)
+    big = int(np.argmax(sizes))
+    small = int(np.argmin(np.where(sizes > 0, sizes, 1 << 30)))
+    t_big = int(np.nonzero((ids == big).any(1))[0][0])
+    t_small = int(np.nonzero((ids == small).any(1))[0][0])
+    n = 8 if cfg.H > 4096 else 24
+    tokens = np.unique(np.concatenate([[0, cfg.T - 1, t_big, t_small],
+                                       rng.choice(cfg.T, n, replace=False)]))
+    ref = _oracle(cfg, hidden, ids, w, weights, tokens=tokens)
+    gu.assert_within_tol(gu.f64(out[torch.from_numpy(tokens).cuda()]), ref,
+                         f"{name} weighted chain")
