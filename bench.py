@@ -599,7 +599,6 @@ FOLD_METRIC = ("down GEMM with the routing weight folded in + combine, ms per la
 def run_fold(args, device, spec) -> dict:
     """Weighted down GEMM + combine on a workload, timed beside the forward's
     own down GEMM (fp32 rows in expert order) + weighted unpermute."""
-    import moe_routed_expert_top_b200 as M
     cfg = get_config(spec["workload"])
     M, layer, hidden, ids, weights, _ = build_layer(cfg, device)
     peaks = load_peaks()
