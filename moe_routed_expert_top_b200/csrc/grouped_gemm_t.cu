@@ -390,7 +390,8 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
             for (int k = 0; k < Cfg::K_STEPS; ++k)
               mma_fp8(d, adesc + 2 * k, bdesc + 2 * k, idesc8, k != 0 ? 1u : 0u);
-            mma_commit(empty0 + 8 * stage);
+            // one commit per K-block: the epilogue, which waits for this
+            // buffer anyway, releases the shared-memory stage when it lands
             mma_commit(tfull0 + 8 * acc);
             if (++stage == STAGES) {
               stage = 0;
@@ -445,6 +446,7 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     int acc = 0;
     uint32_t acc_phase = 0;
+    int stage = 0;  // FP8: the shared-memory stage of the next K-block, as the MMA thread counts
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
       TTile ti;
       if (!t_decode(p, cpre, E, WB, TN, t, ti)) continue;
@@ -488,6 +490,9 @@ __global__ void __launch_bounds__(192, 1)
             ok = false;
             break;
           }
+          // this K-block's MMAs have completed: its shared-memory stage is free
+          if (et == 0) mbar_arrive(empty0 + 8 * stage);
+          if (++stage == STAGES) stage = 0;
           tc_fence_after();
           const uint32_t tbk = lane_base + static_cast<uint32_t>(acc * TN);
           const float4* s4 = reinterpret_cast<const float4*>(sSa + kb * TN);
