@@ -126,3 +126,40 @@ def test_empty_batch_is_a_no_op(M):
     assert L.moe_route_topk(ctypes.byref(p), None, None, None, None) == 0
     assert L.moe_experts_forward(ctypes.byref(p), None, None, None, None, None, None, None, None,
                                  ctypes.c_float(1.0), None, None, ctypes.c_size_t(0), None) == 0
+
+
+def test_weighted_down_and_combine_validation(M):
+    """moe_down_gemm_weighted and moe_combine reject bad arguments on the host,
+    before anything is enqueued, and treat an empty batch as a no-op."""
+    p = M.make_problem(T=16, H=256, F=256, E=8, top_k=2)
+    L = M.lib()
+    f1 = ctypes.c_float(1.0)
+
+    def dw(prob, N=256, K=256, A=16, As=None, B=16, Bs=None, tables=16, w=16, epi=0, y=16, st=16):
+        return L.moe_down_gemm_weighted(ctypes.byref(prob), N, K, A, As, B, Bs, tables, w, f1,
+                                        epi, y, st, None)
+
+    assert dw(p, A=None) == -1
+    assert dw(p, tables=None) == -1
+    assert dw(p, w=None) == -1
+    assert dw(p, st=None) == -1
+    assert dw(p, y=18) == -1                     # misaligned output
+    assert dw(p, epi=M.MOE_EPI_SWIGLU) == -1     # store epilogues only
+    assert dw(p, epi=0x100) == -1                # no gather flag here
+    assert dw(p, epi=M.MOE_TILE_TOKEN_ROWS) == -2
+    assert dw(p, N=192) == -2                    # weight-row tilings need N % 128 == 0
+    assert dw(p, K=96) == -2
+    assert dw(p, As=16) == -1                    # FP8 needs both scale arrays
+    assert dw(M.make_problem(T=16, H=256, F=256, E=8, top_k=2, padding_M=64)) == -2
+    assert dw(M.make_problem(T=0, H=256, F=256, E=8, top_k=2)) == 0
+
+    def cb(prob, y=16, f32=0, tables=16, add=None, out=16):
+        return L.moe_combine(ctypes.byref(prob), y, f32, tables, add, out, None)
+
+    assert cb(p, y=None) == -1
+    assert cb(p, tables=None) == -1
+    assert cb(p, out=None) == -1
+    assert cb(p, out=24) == -1                   # misaligned
+    assert cb(p, add=8) == -1
+    assert cb(M.make_problem(T=16, H=100, F=256, E=8, top_k=2)) == -1   # H % 8
+    assert cb(M.make_problem(T=0, H=256, F=256, E=8, top_k=2)) == 0
