@@ -610,9 +610,62 @@ OPS = {
 for _w in ("qwen3_decode", "qwen3_prefill", "dsv3_prefill", "dsv3_decode_fp8"):
     for _d in ("bf16", "f32"):
         OPS[f"fold_{_w}_{_d}"] = dict(kind="fold", workload=_w, rows=_d)
+# one tensor-parallel rank of the shared expert (moe_shared_expert_forward: the
+# rank's F_s / tp columns of the complete weights, fp32 partial output)
+OPS["shared_kimi_k2_tp1"] = dict(kind="shared", workload="kimi_k2", tp=1)
+OPS["shared_kimi_k2_tp8"] = dict(kind="shared", workload="kimi_k2", tp=8)
+OPS["shared_dsv3_prefill_tp1"] = dict(kind="shared", workload="dsv3_prefill", tp=1)
 OP_METRIC = "training-FP8 op ms + achieved GB/s, % of B200 HBM roofline (1 GPU)"
+SHARED_METRIC = "shared-expert rank partial ms, % of B200 roofline (1 GPU)"
 FOLD_METRIC = ("down GEMM with the routing weight folded in + combine, ms per layer, "
                "% of B200 roofline (1 GPU)")
+
+
+def run_shared(args, device, spec) -> dict:
+    """One rank's shared-expert partial on a workload's tokens: the rank reads its
+    F_s / tp gate, up and down columns of the complete weights in place."""
+    import moe_routed_expert_top_b200 as M
+    cfg = get_config(spec["workload"])
+    tp = spec["tp"]
+    T, H, Fs = cfg.T, cfg.H, cfg.F_shared
+    w = make_weights(cfg, device)
+    wgu, wd = w["ws_gate_up"], w["ws_down"]
+    del w
+    hidden = make_hidden(cfg, device)
+    out = torch.empty(T, H, dtype=torch.float32, device=device)
+    ws = torch.empty(M.moe_shared_workspace_bytes(T, H, Fs, tp), dtype=torch.uint8,
+                     device=device)
+    fn = lambda: M.moe_shared_expert_forward(T, H, Fs, tp, tp - 1, hidden, wgu, wd, True, out, ws)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    peaks = load_peaks()
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0, "device status flag set"
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        ms = statistics.median(time_steps(fn, args.steps, flush, stream))
+    Fp = Fs // tp
+    nbytes = 3 * H * Fp * 2 + T * H * 2 + 2 * T * Fp * 2 + T * H * 4
+    flops = 6.0 * T * H * Fp
+    t_byte = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_flop = flops / (peaks["bf16_tflops"] * 1e12)
+    tensor = t_flop > t_byte
+    achieved = flops / (ms * 1e-3) / 1e12 if tensor else nbytes / (ms * 1e-3) / 1e9
+    peak = peaks["bf16_tflops"] if tensor else peaks["hbm_gbs"]
+    return {
+        "metric": SHARED_METRIC, "op": args.op, "value": round(ms, 4), "unit": "ms",
+        "higher_is_better": False, "steps": args.steps, "warmup": args.warmup, "dtype": "bf16",
+        "data": "synthetic", "config": {"workload": cfg.name, "T": T, "H": H, "F_shared": Fs,
+                                        "tp_size": tp, "tp_rank": tp - 1,
+                                        "l2": "flushed (512 MiB write) before each call"},
+        "roofline": {"bound": "tensor" if tensor else "hbm", "achieved": round(achieved, 1),
+                     "peak": peak, "unit": "TFLOP/s" if tensor else "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "algorithmic_bytes": int(nbytes), "flops": flops},
+        "timing": "median of per-call CUDA events on the launching stream",
+        "clocks": clk.summary(),
+    }
 
 
 def run_fold(args, device, spec) -> dict:
@@ -713,6 +766,8 @@ def run_op(args, device) -> dict:
     spec = dict(OPS[args.op])
     if spec["kind"] == "fold":
         return run_fold(args, device, spec)
+    if spec["kind"] == "shared":
+        return run_shared(args, device, spec)
     if args.override:       # e.g. M=32768: a smaller case of the same op (profiling)
         for item in args.override.split(","):
             key, val = item.split("=", 1)
