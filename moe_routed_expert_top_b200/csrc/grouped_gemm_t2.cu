@@ -636,10 +636,24 @@ bool grouped_gemm_pair_preferred(const GemmLaunch& L) {
 
 cudaError_t launch_grouped_gemm_pair(const GemmLaunch& L, cudaStream_t stream) {
   const bool small = L.group_sizes != nullptr && L.rows <= 64 * L.E;
+  // A dense problem too small to give three quarters of the CTA pairs a
+  // 256-token tile (a tensor-parallel rank's shared expert, few tokens) takes
+  // 128-token tiles: twice the tiles, and the MMA still runs at its full rate
+  // from N = 128 (one rank of tp 8 at Kimi-K2's shared expert: 36 -> 72 tiles).
+  bool mid = false;
+  if (!small && L.group_sizes == nullptr && L.rows > 128) {
+    const long long wb = L.mode == kModeSwiglu ? (L.N / 2) / 128 : L.N / 256;
+    const long long tiles256 = wb * ((static_cast<long long>(L.rows) + 255) / 256);
+    mid = tiles256 * 4 < static_cast<long long>(device_sm_count() / 2) * 3;
+  }
   if (L.mode == kModeSwiglu)
-    return small ? run_pair_g<kPSwiglu, 64>(L, stream) : run_pair_g<kPSwiglu, 256>(L, stream);
+    return small ? run_pair_g<kPSwiglu, 64>(L, stream)
+                 : mid ? run_pair_g<kPSwiglu, 128>(L, stream)
+                       : run_pair_g<kPSwiglu, 256>(L, stream);
   if (L.mode == kModeStore)
-    return small ? run_pair_g<kPStore, 64>(L, stream) : run_pair_g<kPStore, 256>(L, stream);
+    return small ? run_pair_g<kPStore, 64>(L, stream)
+                 : mid ? run_pair_g<kPStore, 128>(L, stream)
+                       : run_pair_g<kPStore, 256>(L, stream);
   return cudaErrorInvalidValue;
 }
 
