@@ -268,8 +268,8 @@ moe_status moe_unpermute(const moe_problem* prob, const float* y, const int32_t*
  *   y_w [P, N], row p = scale * topk_weights[p] * (A @ B[e]^T)[r]
  * i.e. the down GEMM's rows, weighted, in flat pair order p = t*k + j; rows of
  * pairs without a permuted row are not written. `epilogue` = MOE_EPI_STORE
- * (y_w bf16, rounded to nearest even: half the bytes, the rounding of the
- * pages' bf16 y) or MOE_EPI_STORE_F32 (y_w fp32, unrounded), OR-ed with
+ * (y_w bf16, rounded to nearest even: half the bytes, the rounding of the bf16
+ * y that [PR1580]'s unpermute reads) or MOE_EPI_STORE_F32 (y_w fp32, unrounded), OR-ed with
  * MOE_TILE_AUTO, MOE_TILE_WEIGHT_ROWS or MOE_TILE_WEIGHT_ROWS_PAIR and their
  * shape rules (N % 128 == 0; pairs: bf16 operands, N % 256 == 0);
  * MOE_TILE_TOKEN_ROWS: MOE_ERR_UNSUPPORTED. A, A_scales, B, B_scales as for
