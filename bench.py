@@ -33,7 +33,9 @@ sys.path.insert(0, ROOT)
 from moe_inputs import CONFIGS, get_config, make_hidden, make_logits, make_weights  # noqa: E402
 
 METRIC = "routed-experts fwd ms/layer + TFLOPS, % of B200 roofline (1 GPU)"
-DEFAULT_CONFIG = "qwen3_decode"
+# the largest single-GPU workload: DeepSeek-V3-style prefill (T 4096, E 256, k 8,
+# H 7168, F 2048, sigmoid routing, routed_scaling_factor 2.5, shared expert 2048)
+DEFAULT_CONFIG = "dsv3_prefill"
 # TileOPs PR #1580 (H200, bf16) experts-forward times for the same model families
 PAGE_MS = {"qwen3_decode": 3.219, "qwen3_prefill": 6.778, "dsv3_decode_fp8": None,
            "dsv3_prefill": 9.465}
@@ -451,11 +453,7 @@ def run_b200(args, cfg, rank, world, device):
         "vs_baseline": round(ms / page, 4) if page else None,
         "tflops": round(tflops, 2), "dtype": "bf16+e4m3" if cfg.down_fp8 else "bf16",
         "data": "synthetic",
-        "config": {"workload": cfg.name, "T": cfg.T, "E": cfg.E, "top_k": cfg.top_k, "H": cfg.H,
-                   "F": cfg.F, "F_shared": cfg.F_shared, "score_fn": cfg.score_fn,
-                   "routed_scaling_factor": cfg.routed_scaling_factor,
-                   "down_fp8": cfg.down_fp8, "l2": "flushed (512 MiB write) before each step",
-                   "parallelism": f"replicas x{world}"},
+        "config": config_dict(cfg, world),
         "roofline": roof, "forward_roofline": fwd_roof,
         "stages_ms": {k: round(v, 4) for k, v in stages.items()},
         "routing_ms": round(routing_ms, 4),
@@ -484,12 +482,21 @@ def run_b200(args, cfg, rank, world, device):
 # ---------------------------------------------------------------------------
 
 class OracleRunner:
-    """The CPU oracle (as it stands) on the workload: routing and dispatch
-    tables over all tokens, then the per-token expert forward over a sample of
-    tokens. Weights are generated once (seeded N(0, 0.02) bf16 of the
-    workload's shapes; for the DeepSeek-size workloads, whose 22 GB of weights
-    would not fit a host comfortably, each expert the sample touches is drawn
-    when first needed and kept)."""
+    """The CPU oracle (as it stands) on the workload.
+
+    Small workloads run whole: ``O.experts_forward`` over every token. Larger
+    ones run a sample of experts: routing and the dispatch tables over all T
+    tokens, then the oracle's per-expert step (``O.expert_mlp``, which
+    ``experts_forward`` runs once per expert on that expert's rows) over ALL
+    the rows of S seeded experts out of the ``touched`` ones, its time scaled
+    by touched / S; the slot-order weighted sum over the pairs (O(P*H), far
+    below 0.1% of the work) is left out of the timing. Expert weights have the
+    workload's shapes and distribution (seeded N(0, 0.02) bf16, each drawn when
+    first needed and kept; FP8 down weights quantised by the oracle when
+    drawn, like the offline preparation the forward takes as given); drawing
+    them is not timed."""
+
+    FULL_FLOPS = 5e10   # workloads up to this many routed FLOPs run whole
 
     def __init__(self, cfg):
         from oracle import moe_oracle as O
@@ -502,10 +509,13 @@ class OracleRunner:
             self.threads = max([i.get("num_threads", 1) for i in info] + [1])
         except Exception:
             pass
+        self.score = O.SOFTMAX if cfg.score_fn == "softmax" else O.SIGMOID
         self.logits = make_logits(cfg)
         self.hidden = make_hidden(cfg, "cpu")
-        small = cfg.E * cfg.H * cfg.F <= 600_000_000
-        self.weights = make_weights(cfg, "cpu") if small else None
+        self.X = O.as_f64(self.hidden)
+        ids, _ = O.route_topk(self.logits, cfg.top_k, self.score, cfg.renormalize)
+        self.touched = np.unique(ids)
+        self.small = 6.0 * cfg.T * cfg.top_k * cfg.H * cfg.F <= self.FULL_FLOPS
         self.cache = {}
         self.shared = {}
         if cfg.F_shared:
@@ -513,80 +523,123 @@ class OracleRunner:
             self.shared = dict(
                 ws_gate_up=(torch.randn(2 * cfg.F_shared, cfg.H, generator=g) * 0.02).to(torch.bfloat16),
                 ws_down=(torch.randn(cfg.H, cfg.F_shared, generator=g) * 0.02).to(torch.bfloat16))
+        # seeded order in which experts enter the sample
+        self.order = np.random.default_rng(cfg.seed + 99).permutation(self.touched)
 
-    def _loader(self, name, e):
-        if name not in ("w_gate_up", "w_down"):
-            return None
-        key = (name, int(e))
-        if key not in self.cache:
-            g = torch.Generator().manual_seed(2000 + 977 * int(e) + (name == "w_down"))
-            shape = (2 * self.cfg.F, self.cfg.H) if name == "w_gate_up" else (self.cfg.H, self.cfg.F)
-            self.cache[key] = (torch.randn(shape, generator=g) * 0.02).to(torch.bfloat16)
-        return self.cache[key]
+    def _weights(self, e):
+        e = int(e)
+        if e not in self.cache:
+            cfg = self.cfg
+            g = torch.Generator().manual_seed(2000 + 977 * e)
+            wgu = (torch.randn(2 * cfg.F, cfg.H, generator=g) * 0.02).to(torch.bfloat16)
+            wd = (torch.randn(cfg.H, cfg.F, generator=g) * 0.02).to(torch.bfloat16)
+            q = s = None
+            if cfg.down_fp8:
+                w32 = wd.float().numpy()
+                parts = [self.O.quant_weight_128x128(w32[i:i + 512])
+                         for i in range(0, cfg.H, 512)]
+                q = np.concatenate([a for a, _ in parts])
+                s = np.concatenate([b for _, b in parts])
+            self.cache[e] = (wgu, wd, q, s)
+        return self.cache[e]
 
-    def run(self, n: int) -> float:
-        """Seconds for one routed-experts forward of the first n tokens
-        (routing + tables over all T tokens)."""
+    def run(self, S: int):
+        """(seconds of the whole forward, seconds measured) with S sampled experts
+        (all of them on a workload that runs whole)."""
         O, cfg = self.O, self.cfg
+        full = S >= len(self.touched)
+        experts = self.order if full else self.order[:S]
+        for e in experts:
+            self._weights(e)                  # drawn before the timed region
         t0 = time.perf_counter()
-        ids, w = O.route_topk(self.logits, cfg.top_k,
-                              O.SOFTMAX if cfg.score_fn == "softmax" else O.SIGMOID, cfg.renormalize)
+        ids, w = O.route_topk(self.logits, cfg.top_k, self.score, cfg.renormalize)
         O.dispatch_tables(ids, cfg.E, cfg.padding_M)
-        toks = np.arange(n)
-        if self.weights is not None:
-            O.experts_forward(self.hidden, ids, w, self.weights["w_gate_up"], self.weights["w_down"],
-                              cfg.routed_scaling_factor, tokens=toks, fp8=cfg.down_fp8, **self.shared)
-        else:
-            # draw the experts this sample touches (not timed)
-            t_gen = time.perf_counter()
-            for e in np.unique(ids[:n]):
-                self._loader("w_gate_up", e)
-                self._loader("w_down", e)
-            t0 += time.perf_counter() - t_gen
+        t_route = time.perf_counter() - t0
+        if full:
+            def loader(name, e):
+                wgu, wd, q, s = self.cache[int(e)]
+                return {"w_gate_up": wgu, "w_down": wd, "w_down_q": q, "w_down_s": s}[name]
             O.experts_forward(self.hidden, ids, w, None, None, cfg.routed_scaling_factor,
-                              tokens=toks, fp8=cfg.down_fp8, weight_loader=self._loader,
-                              **self.shared)
-        return time.perf_counter() - t0
+                              fp8=cfg.down_fp8, weight_loader=loader, **self.shared)
+            t = time.perf_counter() - t0
+            return t, t
+        t1 = time.perf_counter()
+        flat = ids.reshape(-1)
+        for e in experts:
+            wgu, wd, q, s = self.cache[int(e)]
+            rows = self.X[np.nonzero(flat == e)[0] // cfg.top_k]
+            O.expert_mlp(rows, wgu, wd, fp8=cfg.down_fp8, w_down_q_e=q, w_down_s_e=s)
+        t_mlp = time.perf_counter() - t1
+        t_shared = 0.0
+        if cfg.F_shared:
+            t2 = time.perf_counter()
+            n_sh = max(1, min(cfg.T, 256))
+            O.dense_swiglu_mlp(self.X[:n_sh], self.shared["ws_gate_up"], self.shared["ws_down"])
+            t_shared = (time.perf_counter() - t2) * cfg.T / n_sh
+        measured = time.perf_counter() - t0
+        return t_route + t_mlp * len(self.touched) / len(experts) + t_shared, measured
 
     def pick_sample(self, budget_s: float) -> int:
-        n = min(self.cfg.T, 8)
-        while n < self.cfg.T:
-            if self.run(n) > budget_s / 4:
+        """Experts in the sample: doubled from 2 while one run stays under a quarter
+        of the budget; all of them (the whole workload) for a small one."""
+        if self.small:
+            return len(self.touched)
+        S = 2
+        while S < len(self.touched):
+            _, m = self.run(S)
+            if m * 2 > budget_s / 2:
                 break
-            n = min(self.cfg.T, n * 4)
-        return n
+            S = min(len(self.touched), S * 2)
+        return S
 
-    def describe(self, n: int) -> str:
-        return (f"{n} of {self.cfg.T} tokens through the per-token oracle (all their experts), "
-                f"time scaled by T/{n}; routing + dispatch tables on all {self.cfg.T} tokens")
+    def describe(self, S: int) -> str:
+        cfg = self.cfg
+        if S >= len(self.touched):
+            return (f"the whole workload: routing, dispatch tables and the per-token oracle "
+                    f"forward over all {cfg.T} tokens")
+        d = (f"routing + dispatch tables over all {cfg.T} tokens; the oracle's per-expert "
+             f"step (expert_mlp) over all rows of {S} seeded experts of the "
+             f"{len(self.touched)} touched, time scaled by {len(self.touched)}/{S}")
+        if cfg.F_shared:
+            d += f"; the shared expert over {min(cfg.T, 256)} tokens, scaled by T/{min(cfg.T, 256)}"
+        return d + "; the slot-order weighted sum (O(P*H)) not timed"
 
 
 def cpu_baseline(cfg, budget_s: float = 20.0) -> dict:
     r = OracleRunner(cfg)
-    n = r.pick_sample(budget_s)
-    t = r.run(n)
-    return {"value": round(t * cfg.T / n * 1e3, 1), "unit": "ms/layer", "cores": int(r.threads),
-            "kind": "oracle", "sample": r.describe(n), "sample_s": round(t, 2)}
+    S = r.pick_sample(budget_s)
+    t, m = r.run(S)
+    return {"value": round(t * 1e3, 1), "unit": "ms/layer", "cores": int(r.threads),
+            "kind": "oracle", "sample": r.describe(S), "sample_s": round(m, 2)}
 
 
-def run_reference(args, cfg) -> dict:
+def config_dict(cfg, world: int) -> dict:
+    """The workload as both arms name it."""
+    return {"workload": cfg.name, "T": cfg.T, "E": cfg.E, "top_k": cfg.top_k, "H": cfg.H,
+            "F": cfg.F, "F_shared": cfg.F_shared, "score_fn": cfg.score_fn,
+            "routed_scaling_factor": cfg.routed_scaling_factor, "down_fp8": cfg.down_fp8,
+            "l2": "flushed (512 MiB write) before each step",
+            "parallelism": f"replicas x{world}"}
+
+
+def run_reference(args, cfg, world: int) -> dict:
     r = OracleRunner(cfg)
     per_step = min(20.0, 150.0 / max(1, args.steps + args.warmup))
-    n = r.pick_sample(per_step * 4)
-    times = []
+    S = r.pick_sample(per_step)
+    times, meas = [], []
     for i in range(args.warmup + args.steps):
-        t = r.run(n)
+        t, m = r.run(S)
         if i >= args.warmup:
-            times.append(t * cfg.T / n * 1e3)
+            times.append(t * 1e3)
+            meas.append(m)
     v = round(statistics.median(times), 1)
-    return {"metric": METRIC, "value": v, "unit": "ms/layer", "n_gpus": args.gpus,
+    return {"metric": METRIC, "value": v, "unit": "ms/layer", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": v,
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "impl": "reference",
-            "config": {"workload": cfg.name, "T": cfg.T, "E": cfg.E, "top_k": cfg.top_k,
-                       "H": cfg.H, "F": cfg.F},
+            "data": "synthetic", "impl": "reference", "config": config_dict(cfg, world),
             "cpu_baseline": {"value": v, "unit": "ms/layer", "cores": int(r.threads),
-                             "kind": "oracle", "sample": r.describe(n)},
+                             "kind": "oracle", "sample": r.describe(S),
+                             "sample_s": round(statistics.median(meas), 2)},
             "e2e": {"value": v, "unit": "ms/layer", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
@@ -855,6 +908,21 @@ def max_over_ranks(v: float, world: int, device) -> float:
     return float(t.item())
 
 
+def relaunch_ranks(n: int, argv) -> int:
+    """Start n ranks of this same command, one process per GPU, with the
+    torch.distributed launcher on this node (127.0.0.1), and return its exit
+    status: `python bench.py --gpus N` behaves like the torchrun launch."""
+    import socket
+    with socket.socket() as sock:
+        sock.bind(("127.0.0.1", 0))
+        port = sock.getsockname()[1]
+    args = list(sys.argv[1:] if argv is None else argv)
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n}", "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.abspath(__file__), *args]
+    return subprocess.run(cmd).returncode
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -883,11 +951,16 @@ def main(argv=None):
                  else type(getattr(cfg, k))(v) for k, v in kv.items()}
         cfg = cfg.replace(name=cfg.name + "[" + args.override + "]", **typed)
 
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        return relaunch_ranks(args.gpus, argv)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"bench.py: --gpus {args.gpus} but the launcher started {world} "
+                         f"ranks (WORLD_SIZE); they must agree")
     if args.impl == "reference":
         if rank == 0:
-            print(json.dumps(run_reference(args, cfg)), flush=True)
+            print(json.dumps(run_reference(args, cfg, world)), flush=True)
         return 0
 
     local = int(os.environ.get("LOCAL_RANK", "0"))

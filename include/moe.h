@@ -432,14 +432,45 @@ moe_status moe_gather_rows(int32_t n_dst, int32_t n_src, int64_t row_bytes, cons
  *     the call itself clears what must start at zero (the status word).
  *     Calls whose work overlaps on the GPU (different streams, or different
  *     host threads on one device) race on the array: serialise them.
- *   - The device status word is the array's first int32; it is not readable
- *     through this interface, so device-side flags are not reported here. */
+ *   - The device status word (MOE_DEV_* flags of the last call) is the
+ *     array's first int32; moe_noalloc_read_status copies it out.
+ *   - Argument and shape checks are moe_experts_forward's (T == 0 enqueues
+ *     nothing and touches no device). */
 moe_status moe_experts_forward_noalloc(const moe_problem* prob, const void* hidden,
                                        const int32_t* topk_ids, const float* topk_weights,
                                        const void* w_gate_up, const void* w_down,
                                        const float* w_down_scales,
                                        const void* ws_gate_up, const void* ws_down,
                                        float scale, void* out, moe_stream_t stream);
+
+/* Copies the device status word of the last moe_experts_forward_noalloc call
+ * on the current device (its MOE_DEV_* flags) into *host_status, with one
+ * cudaMemcpyAsync on `stream`. Enqueue it after that call on the same stream;
+ * *host_status is valid once the stream has been synchronised (decode it with
+ * moe_decode_device_status). No counterpart on the pages. Errors: NULL
+ * host_status -> MOE_ERR_INVALID_ARG; a failed CUDA call -> MOE_ERR_CUDA. */
+moe_status moe_noalloc_read_status(int32_t* host_status, moe_stream_t stream);
+
+/* Self-test of the bounded pipeline wait (no counterpart on the pages; the
+ * pages' kernels have no time limits). Every wait on an mbarrier in this
+ * library's kernels gives up after a fixed limit, ORs MOE_DEV_TIMEOUT into the
+ * status word, raises its CTA's abort flag so the CTA's other waiting threads
+ * stop too, drains what it has in flight against one deadline and frees its
+ * tensor memory. This call runs that same wait in a one-CTA kernel on
+ * mbarriers that nothing ever arrives on, with `limit_ns` (1e3 .. 1e9) in place
+ * of the production limit, so a caller can check on its own GPU that a stalled
+ * pipeline ends with a flag and a usable context. The kernel issues no copy
+ * and no MMA. After the stream is synchronised: *dev_status has
+ * MOE_DEV_TIMEOUT set, and dev_result int64 [6] (device memory, 8-byte
+ * aligned) holds {first wait returned true (0 expected), its duration in ns
+ * (>= limit_ns expected), a second thread's wait returned true (0 expected),
+ * its duration in ns (the abort flag ended it, well before its own limit of
+ * 10 * limit_ns), the teardown drain returned true (0 expected), its duration
+ * in ns (>= limit_ns expected)}. The kernel takes about 2 * limit_ns.
+ * Errors: NULL or misaligned pointers, limit_ns out of range ->
+ * MOE_ERR_INVALID_ARG; a launch error -> MOE_ERR_CUDA. */
+moe_status moe_selftest_bounded_wait(int64_t limit_ns, int32_t* dev_status, int64_t* dev_result,
+                                     moe_stream_t stream);
 
 /* Maps a device status word (copied to the host after a sync) to a status:
  * MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_DEVICE_FLAG. */

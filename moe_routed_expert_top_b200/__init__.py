@@ -21,6 +21,7 @@ __all__ = [
     "moe_last_launch_count", "moe_shared_workspace_bytes", "moe_shared_expert_forward",
     "moe_dual_blocks", "moe_quant_dual", "moe_swiglu_quant_dual", "moe_swiglu_backward",
     "moe_ep_split_ids", "moe_gather_rows", "moe_down_gemm_weighted", "moe_combine",
+    "moe_experts_forward_noalloc", "moe_noalloc_read_status", "moe_selftest_bounded_wait",
     "EXPORTED_SYMBOLS",
     "MOE_OK", "MOE_EPI_STORE", "MOE_EPI_SWIGLU", "MOE_EPI_SWIGLU_FP8", "MOE_EPI_STORE_F32",
     "MOE_SCORE_SOFTMAX", "MOE_SCORE_SIGMOID", "MOE_DEV_BAD_EXPERT_ID", "MOE_DEV_TIMEOUT",
@@ -48,6 +49,7 @@ EXPORTED_SYMBOLS = (
     "moe_shared_workspace_bytes", "moe_shared_expert_forward",
     "moe_dual_blocks", "moe_quant_dual", "moe_swiglu_quant_dual", "moe_swiglu_backward",
     "moe_ep_split_ids", "moe_gather_rows", "moe_down_gemm_weighted", "moe_combine",
+    "moe_noalloc_read_status", "moe_selftest_bounded_wait",
 )
 
 
@@ -140,6 +142,8 @@ def lib() -> ctypes.CDLL:
                                             _P, _P, _P]),
         "moe_gather_rows": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int64, _P, _P,
                                            _P, _P, _P]),
+        "moe_noalloc_read_status": (ctypes.c_int, [_P, _P]),
+        "moe_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_int64, _P, _P, _P]),
         "moe_decode_device_status": (ctypes.c_int, [ctypes.c_int32]),
         "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "moe_last_cuda_error": (ctypes.c_char_p, []),
@@ -260,6 +264,31 @@ def moe_experts_forward(prob, hidden, topk_ids, topk_weights, w_gate_up, w_down,
                                      _ptr(w_down_scales), _ptr(ws_gate_up), _ptr(ws_down),
                                      float(scale), _ptr(out), _ptr(workspace), int(ws_bytes),
                                      _stream(stream)), "moe_experts_forward")
+
+
+def moe_experts_forward_noalloc(prob, hidden, topk_ids, topk_weights, w_gate_up, w_down,
+                                w_down_scales, ws_gate_up, ws_down, scale, out, stream=None):
+    _check(lib().moe_experts_forward_noalloc(ctypes.byref(prob), _ptr(hidden), _ptr(topk_ids),
+                                             _ptr(topk_weights), _ptr(w_gate_up), _ptr(w_down),
+                                             _ptr(w_down_scales), _ptr(ws_gate_up), _ptr(ws_down),
+                                             float(scale), _ptr(out), _stream(stream)),
+           "moe_experts_forward_noalloc")
+
+
+def moe_noalloc_read_status(stream=None) -> int:
+    """The status word of the last moe_experts_forward_noalloc call (synchronises
+    the stream to read it)."""
+    import torch
+    v = ctypes.c_int32(-1)
+    _check(lib().moe_noalloc_read_status(ctypes.byref(v), _stream(stream)),
+           "moe_noalloc_read_status")
+    torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
+    return int(v.value)
+
+
+def moe_selftest_bounded_wait(limit_ns, dev_status, dev_result, stream=None):
+    _check(lib().moe_selftest_bounded_wait(int(limit_ns), _ptr(dev_status), _ptr(dev_result),
+                                           _stream(stream)), "moe_selftest_bounded_wait")
 
 
 def moe_shared_workspace_bytes(T, H, F_s, tp_size=1) -> int:

@@ -21,7 +21,7 @@ LIB = os.path.join(PKG, "libmoe_b200.so")
 
 SOURCES = ["api.cu", "grouped_gemm.cu", "grouped_gemm_t.cu", "grouped_gemm_t2.cu",
            "route_permute.cu", "tables.cu", "elementwise.cu", "train_fp8.cu", "ep.cu",
-           "no_alloc.cu"]
+           "no_alloc.cu", "selftest.cu"]
 # translation units whose float32 results must not depend on FMA contraction
 NO_FMA = {"route_permute.cu", "elementwise.cu", "train_fp8.cu"}
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

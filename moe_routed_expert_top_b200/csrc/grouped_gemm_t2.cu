@@ -261,6 +261,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       const CUtensorMap* xmaps[kPXBoxes] = {&tmX0, &tmX1, &tmX2, &tmX3};
       int stage = 0;
       uint32_t phase = 0;
+      uint32_t issued = 0;  // stages whose loads this CTA issued
       bool ok = true;
       for (int t = pair; ok && t < total_tiles; t += npairs) {
         PTile ti;
@@ -316,10 +317,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           if (gather_lane)
             tma_gather4_pair(b_dst + lane * 512, &tmX0, kb * Cfg::BK, g[0], g[1], g[2], g[3], fb,
                              pol_act);
+          ++issued;
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
+        }
+      }
+      if (!ok && lane == 0) {
+        // A wait gave up: the copies of the last min(issued, STAGES) stages may
+        // still be in flight into this CTA's shared memory, completing on the
+        // leader's `full` barriers. The leader waits for those phases (it armed
+        // each with both halves' bytes, so they complete once both CTAs' copies
+        // of the stage have landed); the other CTA cannot wait on the leader's
+        // barriers and instead waits for the MMA's release of each stage on its
+        // own `empty` barriers (a release means both halves landed and were
+        // read). One shared time limit bounds the whole drain; the cluster
+        // barrier at the end keeps both CTAs alive until both have drained.
+        const uint32_t n = issued < static_cast<uint32_t>(STAGES) ? issued : STAGES;
+        const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
+        int s = stage;
+        uint32_t ph = phase;
+        for (uint32_t i = 0; i < n; ++i) {
+          if (--s < 0) {
+            s = STAGES - 1;
+            ph ^= 1u;
+          }
+          if (leader)
+            mbar_wait_until(full0 + 8 * s, ph, deadline);
+          else
+            mbar_wait_until(empty0 + 8 * s, ph, deadline);
         }
       }
       // every load this CTA issued has been consumed (its stage released) before leaving

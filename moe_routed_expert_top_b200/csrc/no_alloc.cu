@@ -53,12 +53,14 @@ extern "C" moe_status moe_experts_forward_noalloc(const moe_problem* prob, const
                                                   const float* w_down_scales,
                                                   const void* ws_gate_up, const void* ws_down,
                                                   float scale, void* out, moe_stream_t stream) {
-  if (prob == nullptr) return MOE_ERR_INVALID_ARG;
-  if (prob->T == 0) return MOE_OK;
-  const size_t need = moe_workspace_bytes(prob);
-  if (need == 0) return MOE_ERR_UNSUPPORTED;
   // too large for the built-in scratch area: rejected before anything is enqueued
+  const size_t need = moe_workspace_bytes(prob);  // 0 for a problem the forward rejects
   if (need > static_cast<size_t>(MOE_NOALLOC_SCRATCH_BYTES)) return MOE_ERR_WORKSPACE;
+  // an invalid problem, or T == 0: moe_experts_forward decides the status
+  // (check_problem's error, or MOE_OK with nothing enqueued) without the device
+  if (need == 0 || prob->T == 0)
+    return moe_experts_forward(prob, hidden, topk_ids, topk_weights, w_gate_up, w_down,
+                               w_down_scales, ws_gate_up, ws_down, scale, out, nullptr, 0, stream);
   cudaError_t err = cudaSuccess;
   void* ws = scratch_for_current_device(&err);
   if (ws == nullptr) return MOE_ERR_CUDA;
@@ -67,4 +69,15 @@ extern "C" moe_status moe_experts_forward_noalloc(const moe_problem* prob, const
   return moe_experts_forward(prob, hidden, topk_ids, topk_weights, w_gate_up, w_down,
                              w_down_scales, ws_gate_up, ws_down, scale, out, ws,
                              static_cast<size_t>(MOE_NOALLOC_SCRATCH_BYTES), stream);
+}
+
+extern "C" moe_status moe_noalloc_read_status(int32_t* host_status, moe_stream_t stream) {
+  if (host_status == nullptr) return MOE_ERR_INVALID_ARG;
+  cudaError_t err = cudaSuccess;
+  void* ws = scratch_for_current_device(&err);
+  if (ws == nullptr) return MOE_ERR_CUDA;
+  // the status word is the first int32 of the forward's workspace
+  err = cudaMemcpyAsync(host_status, ws, sizeof(int32_t), cudaMemcpyDeviceToHost,
+                        reinterpret_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -68,17 +68,17 @@ constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s
 
 // Bounded wait for the phase with `parity` to complete. Returns false (after
 // OR-ing MOE_DEV_TIMEOUT into *status and raising the CTA's abort flag) if the
-// time limit passes, or immediately if another thread of the CTA already
-// aborted.
+// time limit (default kWaitLimitNs) passes, or soon after another thread of
+// the CTA raised the abort flag.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int32_t* status) {
+                                          int32_t* status, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0u) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         if (status) atomicOr(status, MOE_DEV_TIMEOUT_FLAG);
         return false;
@@ -94,6 +94,15 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 255u && globaltimer_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+
+// The same against an absolute %globaltimer deadline, so that a drain over
+// several barriers shares one time limit.
+__device__ __forceinline__ bool mbar_wait_until(uint32_t bar, uint32_t parity, uint64_t deadline) {
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 255u && globaltimer_ns() > deadline) return false;
   }
 }
 

@@ -144,7 +144,15 @@ class SharedFusedMoE:
                 world_size: int = 1) -> torch.Tensor:
         """bf16(all_reduce_sum(shared_partial) + routed_out): the caller's side
         of the contract (``group``/``world_size`` of the tensor-parallel ranks;
-        no collective when world_size == 1)."""
+        no collective when world_size == 1).
+
+        Rounding: ``routed_out`` is already one bf16 rounding of the routed sum
+        (moe_experts_forward's output), and this add rounds once more, as the
+        pages' contract adds two tensors (TileOPs PR #778, Partial output
+        contract). The one-GPU path with ``F_shared > 0`` instead adds the
+        shared expert in fp32 before its single cast. The two differ by at
+        most one bf16 rounding of the routed part (2**-9 relative), inside the
+        forward's tolerance."""
         if shared_partial is None:
             return routed_out
         if world_size > 1:

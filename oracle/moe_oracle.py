@@ -593,9 +593,9 @@ def unpermute(y: np.ndarray, row_of_pair: np.ndarray, topk_weights: np.ndarray,
 def weighted_rows(y: np.ndarray, pair_of_row: np.ndarray, topk_weights: np.ndarray,
                   scale: float, round_output: bool = True):
     """The down projection's rows with the routing weight and scale applied,
-    moved to flat pair order (SURVEY's "fold the routing weight x scale into
-    the down-GEMM epilogue": TileOPs PR #1580 §Unpermute's scale folding done
-    one step earlier, as a per-row scale x routing weight):
+    moved to flat pair order (the routing weight x scale folded into the
+    down-GEMM epilogue: TileOPs PR #1580 §Unpermute's scale folding done one
+    step earlier, as pypto-lib PR #809's per-row scale x routing weight):
         y_w[p] = bf16( scale * w[p] * y[r] )   for every row r with p = pair_of_row[r] >= 0
     The bf16 rounding is the one the pages put on the down GEMM's output (y is
     bf16 [P, H] in their layout); ``round_output=False`` keeps the float64

@@ -163,3 +163,38 @@ def test_weighted_down_and_combine_validation(M):
     assert cb(p, add=8) == -1
     assert cb(M.make_problem(T=16, H=100, F=256, E=8, top_k=2)) == -1   # H % 8
     assert cb(M.make_problem(T=0, H=256, F=256, E=8, top_k=2)) == 0
+
+
+def test_noalloc_validates_like_the_workspace_forward(M):
+    """moe_experts_forward_noalloc leaves every argument and shape check to
+    moe_experts_forward: an invalid problem gets that call's status even at
+    T = 0, a valid T = 0 problem is a no-op that touches no device, and a
+    problem too large for the built-in scratch array is MOE_ERR_WORKSPACE."""
+    L = M.lib()
+    f1 = ctypes.c_float(1.0)
+
+    def na(prob):
+        return L.moe_experts_forward_noalloc(ctypes.byref(prob), None, None, None, None, None,
+                                             None, None, None, f1, None, None)
+
+    assert L.moe_experts_forward_noalloc(None, None, None, None, None, None, None, None, None,
+                                         f1, None, None) == M.MOE_ERR_INVALID_ARG
+    for kw, status in ((dict(E=0), -1), (dict(E=1025), -2), (dict(top_k=9, E=8), -2),
+                       (dict(H=100), -2), (dict(score_fn=7), -1)):
+        base = dict(T=0, H=256, F=256, E=8, top_k=2)
+        base.update(kw)
+        assert na(M.make_problem(**base)) == status, kw
+    assert na(M.make_problem(T=0, H=256, F=256, E=8, top_k=2)) == M.MOE_OK
+    big = M.make_problem(T=4096, H=2048, F=768, E=128, top_k=8)
+    assert M.moe_workspace_bytes(big) > 64 * 1024 * 1024
+    assert na(big) == M.MOE_ERR_WORKSPACE
+    assert L.moe_noalloc_read_status(None, None) == M.MOE_ERR_INVALID_ARG
+
+
+def test_selftest_bounded_wait_validation(M):
+    L = M.lib()
+    assert L.moe_selftest_bounded_wait(1000000, None, 16, None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_selftest_bounded_wait(1000000, 16, None, None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_selftest_bounded_wait(1000000, 16, 20, None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_selftest_bounded_wait(999, 16, 16, None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_selftest_bounded_wait(2000000000, 16, 16, None) == M.MOE_ERR_INVALID_ARG

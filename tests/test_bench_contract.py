@@ -32,3 +32,30 @@ def test_reference_arm_line_has_the_contract_keys():
     e2e = d["e2e"]
     assert e2e["value"] == d["value"] and e2e["unit"] == d["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+def test_gpus_flag_starts_that_many_ranks():
+    """`python bench.py --gpus 2` (no launcher) starts two ranks itself through
+    the torch.distributed launcher; rank 0 alone prints the line, and it
+    reports n_gpus 2 (the reference arm on the tiny workload, on the CPU)."""
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2",
+                        "--impl", "reference", "--config", "tiny", "--steps", "1",
+                        "--warmup", "3"], capture_output=True, text=True, cwd=ROOT,
+                       timeout=600, env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    assert d["n_gpus"] == 2 and d["impl"] == "reference"
+    assert d["config"]["parallelism"] == "replicas x2"
+
+
+def test_gpus_flag_must_match_the_launchers_world_size():
+    env = dict(os.environ, WORLD_SIZE="2", RANK="1", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "1",
+                        "--impl", "reference", "--config", "tiny", "--steps", "1"],
+                       capture_output=True, text=True, cwd=ROOT, timeout=600, env=env)
+    assert r.returncode != 0
+    assert "must agree" in r.stderr

@@ -6,8 +6,10 @@ Shapes span several M-, N- and K-tiles, ragged expert tails, empty experts and
 experts of 1/127/128/129 rows. Tolerance for bf16 outputs: |err| <= 1e-2 +
 1e-2*|ref|; fp32 outputs 1e-4 + 1e-4*|ref|. FP8 codes and scales: bit-exact
 against the oracle when the oracle's fp32 h is fed to the quantiser; the fused
-epilogue's codes are checked against the oracle's h by the E4M3 error bound and
-byte-for-byte against the standalone quantiser on the same h."""
+epilogue's codes and scales bit for bit against the oracle's quantiser fed the
+kernel's own fp32 h (also at the full DeepSeek-V3 decode size, in the launch
+configuration the benchmark times), and against the oracle's h by the E4M3
+error bound."""
 import numpy as np
 import pytest
 import torch
@@ -218,8 +220,13 @@ def test_grouped_gemm_swiglu_fp8_epilogue(T, E, k, H, F, sizes):
     deq = O.e4m3_value(q.cpu().numpy()) * np.repeat(s.cpu().numpy().astype(np.float64), 128, 1)
     bound = np.abs(h_ref) * (2.0 ** -4 + 2e-3) + np.repeat(amax / 448, 128, 1) * (2.0 ** -9 + 1e-3)
     assert np.all(np.abs(deq - h_ref) <= bound)
+    # bit for bit against the oracle's quantiser fed the kernel's own fp32 h
+    # (XTuner PR #2089 review thread: bitwise tests of the fused kernel)
+    q_ref, s_ref = O.quant_1x128(dh.cpu().numpy())
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
     # the fused epilogue and the standalone quantiser agree byte for byte on the
-    # same fp32 h (the standalone one is bit-exact against the oracle)
+    # same fp32 h
     q2 = torch.zeros_like(q)
     s2 = torch.zeros_like(s)
     M.moe_swiglu_quant(P, F, None, dh, 1, q2, s2)
@@ -380,3 +387,32 @@ def test_weight_quant_bit_exact():
         rq, rs = O.quant_weight_128x128(gu.f64(w[e]).astype(np.float32))
         assert np.array_equal(q[e].cpu().numpy(), rq)
         assert np.array_equal(s[e].cpu().numpy().view(np.uint32), rs.view(np.uint32))
+
+
+def test_swiglu_fp8_epilogue_full_size_bits():
+    """The fused SwiGLU + 1x128 FP8 epilogue on the DeepSeek-V3 decode workload
+    (T 512, E 256, k 8, H 7168, F 2048, skewed routing): every code and scale
+    equals the oracle's quantiser applied to the kernel's own fp32 h."""
+    gu = _gu()
+    import moe_routed_expert_top_b200 as M
+    from moe_inputs import make_hidden, make_logits, make_weights
+    cfg = get_config("dsv3_decode_fp8")
+    ids, _ = O.route_topk(make_logits(cfg), cfg.top_k, gu.score_code(cfg), cfg.renormalize)
+    hidden = make_hidden(cfg, "cuda")
+    weights = make_weights(cfg, "cuda")
+    wgu = weights.pop("w_gate_up")
+    del weights
+    L, tables, status, x_perm = gu.gpu_tables(cfg, ids, hidden=hidden)
+    prob = gu.problem(cfg)
+    P, F = L["P"], cfg.F
+    q = torch.zeros(P, F, dtype=torch.uint8, device="cuda")
+    sc = torch.zeros(P, F // 128, dtype=torch.float32, device="cuda")
+    dh = torch.zeros(P, F, dtype=torch.float32, device="cuda")
+    M.moe_grouped_gemm(prob, 0, 2 * F, cfg.H, x_perm, None, wgu, None, tables,
+                       M.MOE_EPI_SWIGLU_FP8, q, sc, dh, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    q_ref, s_ref = O.quant_1x128(dh.cpu().numpy())
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(sc.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert (s_ref > 0).all()

@@ -1,10 +1,14 @@
 """GPU test of moe_experts_forward_noalloc, the forward for callers that cannot
 allocate device memory (its workspace is a fixed 64 MiB array inside the
 library). Called through the C ABI twice in a row, its output must match the
-regular moe_experts_forward (caller-supplied workspace) within the bf16
-tolerance used by every forward test; a problem too large for the array is
-rejected before anything runs. Collected last so a failure here comes after
-every other test has run; it also passes alone in a fresh process."""
+CPU oracle (every element of the small case, seeded token samples of the
+decode workload) and the regular moe_experts_forward (caller-supplied
+workspace), within the bf16 tolerance used by every forward test; its status
+word, read back with moe_noalloc_read_status, is 0 after a clean call and
+carries MOE_DEV_BAD_EXPERT_ID after a call with an out-of-range expert id; a
+problem too large for the array is rejected before anything runs. Collected
+last so a failure here comes after every other test has run; it also passes
+alone in a fresh process."""
 import ctypes
 
 import numpy as np
@@ -30,8 +34,14 @@ def _noalloc(M, prob, hidden, ids, w, wgu, wd, scale, out):
                                          torch.cuda.current_stream().cuda_stream)
 
 
+def _oracle(cfg, hidden, ids, w, weights, tokens):
+    loader = lambda name, e: weights[name][e].float().cpu()
+    return O.experts_forward(hidden.float().cpu(), ids, w, None, None,
+                             cfg.routed_scaling_factor, tokens=tokens, weight_loader=loader)
+
+
 @pytest.mark.parametrize("cfg", CASES, ids=[c.name for c in CASES])
-def test_noalloc_matches_workspace_forward_twice(cfg):
+def test_noalloc_matches_oracle_and_workspace_forward_twice(cfg):
     from moe_routed_expert_top_b200 import build
     build.build()
     import moe_routed_expert_top_b200 as M
@@ -44,6 +54,13 @@ def test_noalloc_matches_workspace_forward_twice(cfg):
                                 O.SOFTMAX if cfg.score_fn == "softmax" else O.SIGMOID, True)
     ids = torch.from_numpy(ids_np).cuda()
     w = torch.from_numpy(w_np).cuda()
+    # the oracle on every token of the small case, on a seeded sample of the decode one
+    if cfg.T <= 256:
+        tokens = np.arange(cfg.T)
+    else:
+        tokens = np.unique(np.concatenate([[0, cfg.T - 1], np.random.default_rng(3).choice(
+            cfg.T, 64, replace=False)]))
+    oracle = _oracle(cfg, hidden, ids_np, w_np, weights, tokens)
     ref = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device="cuda")
     ws = torch.empty(M.moe_workspace_bytes(prob), dtype=torch.uint8, device="cuda")
     M.moe_experts_forward(prob, hidden, ids, w, weights["w_gate_up"], weights["w_down"], None,
@@ -56,8 +73,32 @@ def test_noalloc_matches_workspace_forward_twice(cfg):
                       cfg.routed_scaling_factor, out)
         assert st == 0, M.moe_status_string(st)
         torch.cuda.synchronize()
-        assert_within_tol(out.double().cpu().numpy(), ref_np, f"noalloc {cfg.name}")
-        assert np.isfinite(out.double().cpu().numpy()).all()
+        got = out.double().cpu().numpy()
+        assert np.isfinite(got).all()
+        assert_within_tol(got[tokens], oracle, f"noalloc vs oracle {cfg.name}")
+        assert_within_tol(got, ref_np, f"noalloc vs workspace forward {cfg.name}")
+        assert M.moe_noalloc_read_status() == 0
+
+
+def test_noalloc_status_word_reports_bad_expert_id():
+    from moe_routed_expert_top_b200 import build
+    build.build()
+    import moe_routed_expert_top_b200 as M
+    from tests.gpu_util import problem, random_ids
+    cfg = get_config("tiny", name="noalloc_flag", T=64, E=8, top_k=2, H=256, F=128, seed=42)
+    prob = problem(cfg)
+    weights = make_weights(cfg, "cuda")
+    hidden = make_hidden(cfg, "cuda")
+    ids_np = random_ids(cfg.T, cfg.E, cfg.top_k, np.random.default_rng(6))
+    w = torch.full((cfg.T, cfg.top_k), 0.5, dtype=torch.float32, device="cuda")
+    out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device="cuda")
+    bad = ids_np.copy()
+    bad[5, 1] = cfg.E          # one pair routed outside [0, E): skipped and flagged
+    for ids_case, flag in ((bad, M.MOE_DEV_BAD_EXPERT_ID), (ids_np, 0)):
+        ids = torch.from_numpy(ids_case).cuda()
+        st = _noalloc(M, prob, hidden, ids, w, weights["w_gate_up"], weights["w_down"], 1.0, out)
+        assert st == 0, M.moe_status_string(st)
+        assert M.moe_noalloc_read_status() == flag
 
 
 def test_noalloc_rejects_problem_larger_than_its_scratch():
