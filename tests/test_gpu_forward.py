@@ -105,17 +105,10 @@ def test_forward_all_elements(cfg):
     gu.assert_within_tol(gu.f64(out), ref, cfg.name)
 
 
-@pytest.mark.parametrize("name", [n for n in CONFIGS if n != "tiny"])
-def test_forward_full_size_sampled(name):
-    gu = _gu()
-    cfg = get_config(name)
-    hidden, ids, w, weights = _inputs(cfg)
-    out, _ = _run(cfg, hidden, ids, w, weights)
+def _sample_tokens(cfg, ids, n):
+    """>= n seeded tokens, including tokens routed to the most and to the least
+    loaded experts and the first and last token."""
     rng = np.random.default_rng(7)
-    # >= 256 seeded tokens (the Kimi-K2-size layer, 384 experts plus an 18432-wide
-    # shared expert, a smaller sample), including tokens routed to the most and
-    # to the least loaded experts
-    n = 24 if cfg.name == "kimi_k2" else 256
     sizes = np.bincount(ids.reshape(-1), minlength=cfg.E)
     big = int(np.argmax(sizes))
     small = int(np.argmin(np.where(sizes > 0, sizes, 1 << 30)))
@@ -124,6 +117,18 @@ def test_forward_full_size_sampled(name):
     tokens = np.unique(np.concatenate([[0, cfg.T - 1], t_big, t_small,
                                        rng.choice(cfg.T, n, replace=False)]))
     assert len(tokens) >= min(n, cfg.T)
+    return tokens
+
+
+@pytest.mark.parametrize("name", [n for n in CONFIGS if n != "tiny" and not CONFIGS[n].down_fp8])
+def test_forward_full_size_sampled(name):
+    gu = _gu()
+    cfg = get_config(name)
+    hidden, ids, w, weights = _inputs(cfg)
+    out, _ = _run(cfg, hidden, ids, w, weights)
+    # >= 256 seeded tokens (the Kimi-K2-size layer, 384 experts plus an 18432-wide
+    # shared expert, a smaller sample)
+    tokens = _sample_tokens(cfg, ids, 24 if cfg.name == "kimi_k2" else 256)
     ref = _oracle(cfg, hidden, ids, w, weights, tokens=tokens)
     gu.assert_within_tol(gu.f64(out[torch.from_numpy(tokens).cuda()]), ref, name)
     assert torch.isfinite(out.float()).all()
@@ -179,3 +184,114 @@ def test_deterministic_repeat():
     b = layer.forward(hidden, torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda())
     torch.cuda.synchronize()
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_shared_expert_in_the_routed_launch():
+    """A workload whose routed gate+up GEMM is weight-bound and whose shared
+    expert is compute-bound: the shared gate+up runs in the same pair-kernel
+    launch as the routed one, on pairs of its own (one launch fewer), and every
+    output element matches the oracle."""
+    import moe_routed_expert_top_b200 as M
+    gu = _gu()
+    cfg = get_config("tiny", name="shared_dual", T=1024, E=16, top_k=2, H=2048, F=1024,
+                     score_fn="sigmoid", routed_scaling_factor=2.5, F_shared=2048, seed=24)
+    hidden, ids, w, weights = _inputs(cfg)
+    out, _ = _run(cfg, hidden, ids, w, weights)
+    # tables (2) + gather + gate+up with the shared gate+up + routed down +
+    # shared down + unpermute
+    assert M.moe_last_launch_count() == 7
+    ref = _oracle(cfg, hidden, ids, w, weights)
+    gu.assert_within_tol(gu.f64(out), ref, cfg.name)
+
+
+def test_shared_expert_launches_on_the_headline_workload():
+    """DeepSeek-V3 prefill: both shared GEMMs share their routed counterpart's
+    launch (tables 2, gather, gate+up, down, unpermute)."""
+    import moe_routed_expert_top_b200 as M
+    cfg = get_config("dsv3_prefill")
+    hidden, ids, w, weights = _inputs(cfg)
+    _run(cfg, hidden, ids, w, weights)
+    assert M.moe_last_launch_count() == 6
+
+
+@pytest.mark.parametrize("name", [n for n in CONFIGS if CONFIGS[n].down_fp8])
+def test_forward_fp8_full_size_sampled(name):
+    """The FP8 forward at full size on >= 256 seeded tokens, step by step
+    against the oracle.
+
+    E4M3 codes are a discontinuous function of h: the GPU's h (fp32 tensor-core
+    sums over K = 7168) and the oracle's (float64 sums) differ by ~1e-5 of the
+    row's largest value, and a code whose h/s sits that close to an E4M3
+    rounding midpoint comes out one step apart on the two sides (about 4 in
+    10^4 codes here). One such step at a tile's largest value moves the whole
+    output row of its token by up to ~0.03. So:
+      (1) the fused gate+up + SwiGLU h agrees with the oracle's h within 1e-4
+          of the row's largest |h|, and its codes and scales are the oracle's
+          quantiser applied to that h, bit for bit;
+      (2) the rest of the path -- the FP8 block-scaled down GEMM in the
+          forward's launch configuration and the weighted unpermute -- fed the
+          ORACLE's codes and scales, meets max |err| <= 1e-2 + 1e-2*|ref|
+          against the oracle's output on every sampled element;
+      (3) end to end (each side quantising its own h), at most 0.1% of the
+          sampled outputs lie outside that tolerance, none beyond 4x it."""
+    gu = _gu()
+    import moe_routed_expert_top_b200 as M
+    cfg = get_config(name)
+    hidden, ids, w, weights = _inputs(cfg)
+    out, layer = _run(cfg, hidden, ids, w, weights)
+    tokens = _sample_tokens(cfg, ids, 256)
+    P, F, H, k = cfg.T * cfg.top_k, cfg.F, cfg.H, cfg.top_k
+    L, tables, status, x_perm = gu.gpu_tables(cfg, ids, hidden=hidden)
+    rop = gu.split_tables(L, tables, cfg.E)["row_of_pair"]
+    prob = gu.problem(cfg)
+    q = torch.zeros(P, F, dtype=torch.uint8, device="cuda")
+    sc = torch.zeros(P, F // 128, dtype=torch.float32, device="cuda")
+    dh = torch.zeros(P, F, dtype=torch.float32, device="cuda")
+    M.moe_grouped_gemm(prob, 0, 2 * F, H, x_perm, None, weights["w_gate_up"], None, tables,
+                       M.MOE_EPI_SWIGLU_FP8, q, sc, dh, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    h_gpu = dh.cpu().numpy()
+    q_gpu, s_gpu = q.cpu().numpy(), sc.cpu().numpy()
+    # the oracle, expert by expert over the sampled tokens' pairs, keeping its
+    # own h, codes and scales
+    X = gu.f64(hidden)
+    sub = ids[tokens]
+    qa_all = np.zeros((P, F), np.uint8)
+    sa_all = np.zeros((P, F // 128), np.float32)
+    acc = np.zeros((len(tokens), H))
+    for e in np.unique(sub):
+        ti, ji = np.nonzero(sub == e)
+        wq_e, ws_e = _oracle_weight_fp8(weights["w_down"][e])
+        y, parts = O.expert_mlp(X[tokens[ti]], weights["w_gate_up"][e].float().cpu(), None,
+                                fp8=True, w_down_q_e=wq_e, w_down_s_e=ws_e, return_parts=True)
+        rows = rop[tokens[ti] * k + ji]
+        # (1) h within 1e-4 of the row's largest |h|; codes of the GPU's h
+        hr = parts["h"]
+        tol_h = 1e-4 * np.abs(hr).max(1, keepdims=True)
+        assert np.all(np.abs(h_gpu[rows] - hr) <= tol_h), f"h of expert {e}"
+        qa_all[rows], sa_all[rows] = parts["q"], parts["sa"]
+        np.add.at(acc, ti, w[tokens[ti], ji][:, None] * y)
+    ref = O.bf16_round(cfg.routed_scaling_factor * acc)
+    q_ref, s_ref = O.quant_1x128(h_gpu)
+    assert np.array_equal(q_gpu, q_ref)
+    assert np.array_equal(s_gpu.view(np.uint32), s_ref.view(np.uint32))
+    # (2) the down GEMM + unpermute fed the oracle's codes and scales
+    y = torch.empty(P, H, dtype=torch.float32, device="cuda")
+    M.moe_grouped_gemm(prob, 0, H, F, torch.from_numpy(qa_all).cuda(),
+                       torch.from_numpy(sa_all).cuda(), layer.w_down, layer.w_down_scales, tables,
+                       M.MOE_EPI_STORE_F32, y, None, None, status)
+    out2 = torch.empty(cfg.T, H, dtype=torch.bfloat16, device="cuda")
+    M.moe_unpermute(prob, y, tables, torch.from_numpy(w).cuda(), cfg.routed_scaling_factor,
+                    None, out2)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    gu.assert_within_tol(gu.f64(out2)[tokens], ref, f"{name}: down + unpermute on oracle codes")
+    # (3) end to end
+    got = gu.f64(out)[tokens]
+    err = np.abs(got - ref)
+    bound = 1e-2 + 1e-2 * np.abs(ref)
+    frac = float((err > bound).mean())
+    assert frac <= 1e-3, frac
+    assert np.all(err <= 4 * bound), float((err / bound).max())
+    assert torch.isfinite(out.float()).all()
