@@ -105,7 +105,7 @@ enum {
  *   MOE_TILE_WEIGHT_ROWS 128 weight rows x (the expert's tokens, <= 256, rounded
  *                        up to 16) per tile: MMA work follows the real group
  *                        sizes; MOE_EPI_STORE / STORE_F32 (N % 128 == 0; in
- *                        FP8 mode also K <= 4096) or bf16 MOE_EPI_SWIGLU
+ *                        FP8 mode also K <= 2048) or bf16 MOE_EPI_SWIGLU
  *                        (N % 128 == 0) only, else MOE_ERR_UNSUPPORTED.
  *   MOE_TILE_WEIGHT_ROWS_PAIR  256 weight rows x (tokens, <= 256) per tile,
  *                        computed by two CTAs of a cluster with one 256-row
@@ -274,7 +274,7 @@ moe_status moe_unpermute(const moe_problem* prob, const float* y, const int32_t*
  * shape rules (N % 128 == 0; pairs: bf16 operands, N % 256 == 0);
  * MOE_TILE_TOKEN_ROWS: MOE_ERR_UNSUPPORTED. A, A_scales, B, B_scales as for
  * moe_grouped_gemm's store epilogues (bf16, or FP8 block-scaled with
- * K <= 4096); tables as written by moe_route_permute (padding_M 128);
+ * K <= 2048); tables as written by moe_route_permute (padding_M 128);
  * topk_weights fp32 [T, k]. Device flags: MOE_DEV_TIMEOUT into *dev_status
  * (required). */
 moe_status moe_down_gemm_weighted(const moe_problem* prob, int32_t N, int32_t K, const void* A,

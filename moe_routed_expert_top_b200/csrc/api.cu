@@ -446,38 +446,7 @@ moe_status moe_experts_forward(const moe_problem* prob, const void* hidden,
   MOE_CUDA_TRY(moe::launch_gather_rows(hidden, tables + L.pair_of_row, L.P, k, H, x_perm, st));
   g_last_launches += 1;
   g.A = x_perm;
-
-  // the shared expert: a dense SwiGLU MLP on all tokens, added in the unpermute
-  // (TileOPs PR #778, Design). Its GEMMs are compute-bound while the routed
-  // experts' are weight-bound, so where both take the same pair-kernel shape
-  // each shared GEMM runs in the same launch as its routed counterpart, on a
-  // few SM pairs of its own.
-  moe::GemmLaunch d;
-  const float* addend = nullptr;
-  if (prob->F_shared > 0) {
-    d.rows = T;
-    d.E = 1;
-    d.status = status;
-    d.mode = moe::kModeSwiglu;
-    d.N = 2 * prob->F_shared;
-    d.K = H;
-    d.A = hidden;
-    d.B = ws_gate_up;
-    d.C = base + w.hs;
-    addend = reinterpret_cast<const float*>(base + w.ys);
-  }
-  bool fused = false;
-  if (prob->F_shared > 0) MOE_CUDA_TRY(moe::launch_grouped_gemm_pair_dual(g, d, st, &fused));
-  if (fused) {
-    g_last_launches += 1;
-  } else {
-    MOE_CUDA_TRY(moe::launch_grouped_gemm(g, st));
-    g_last_launches += 1;
-    if (prob->F_shared > 0) {
-      MOE_CUDA_TRY(moe::launch_grouped_gemm(d, st));
-      g_last_launches += 1;
-    }
-  }
+  MOE_CUDA_TRY(moe::launch_grouped_gemm(g, st));
   // a6: down, fp32 rows in expert order for the weighted unpermute. (Folding
   // the routing weight into this epilogue, moe_down_gemm_weighted, writes the
   // rows in flat pair order: in fp32 that measured as fast on DeepSeek shapes
@@ -494,7 +463,23 @@ moe_status moe_experts_forward(const moe_problem* prob, const void* hidden,
   g.C = y;
   g.out_f32 = 1;
   g.C_scales = nullptr;
+  MOE_CUDA_TRY(moe::launch_grouped_gemm(g, st));
+  g_last_launches += 2;
+
+  // shared expert: a dense SwiGLU MLP on all tokens, added in the unpermute
+  const float* addend = nullptr;
   if (prob->F_shared > 0) {
+    moe::GemmLaunch d;
+    d.rows = T;
+    d.E = 1;
+    d.status = status;
+    d.mode = moe::kModeSwiglu;
+    d.N = 2 * prob->F_shared;
+    d.K = H;
+    d.A = hidden;
+    d.B = ws_gate_up;
+    d.C = base + w.hs;
+    MOE_CUDA_TRY(moe::launch_grouped_gemm(d, st));
     d.mode = moe::kModeStore;
     d.N = H;
     d.K = prob->F_shared;
@@ -502,18 +487,9 @@ moe_status moe_experts_forward(const moe_problem* prob, const void* hidden,
     d.B = ws_down;
     d.C = base + w.ys;
     d.out_f32 = 1;
-  }
-  fused = false;
-  if (prob->F_shared > 0) MOE_CUDA_TRY(moe::launch_grouped_gemm_pair_dual(g, d, st, &fused));
-  if (fused) {
-    g_last_launches += 1;
-  } else {
-    MOE_CUDA_TRY(moe::launch_grouped_gemm(g, st));
-    g_last_launches += 1;
-    if (prob->F_shared > 0) {
-      MOE_CUDA_TRY(moe::launch_grouped_gemm(d, st));
-      g_last_launches += 1;
-    }
+    MOE_CUDA_TRY(moe::launch_grouped_gemm(d, st));
+    addend = reinterpret_cast<const float*>(base + w.ys);
+    g_last_launches += 2;
   }
   // a7
   MOE_CUDA_TRY(moe::launch_unpermute(y, tables + L.row_of_pair, topk_weights, T, k, H, scale,

@@ -84,12 +84,17 @@ struct TCfg {
   // 32 token rows x 128 fp32, then the tile's row destinations and factors
   // (weighted store)
   static constexpr int STAGE_OUT_BYTES = 32 * 128 * 4 + 2 * TN * 4;
-  static constexpr int MAX_KBS = 32;                    // FP8: K <= 4096
-  static constexpr int SA_BYTES = kFp8 ? TN * MAX_KBS * 4 : 0;
-  static constexpr int NUM_BARS = 2 * STAGES + 2 * NUM_ACC + 1;
+  // FP8: a scale warp (warp 6) prepares each tile's sa * sw products one tile
+  // ahead in a ring of two slots of TN x MAX_KBS fp32
+  static constexpr int kThreads = kFp8 ? 224 : 192;
+  static constexpr int MAX_KBS = 16;                    // FP8: K <= 2048
+  static constexpr int SA_SLOT = TN * MAX_KBS;          // floats per slot
+  static constexpr int SA_BYTES = kFp8 ? 2 * SA_SLOT * 4 : 0;
+  static constexpr int NUM_BARS = 2 * STAGES + 2 * NUM_ACC + 1 + (kFp8 ? 4 : 0);
   static constexpr int MAX_E = 1024;
+  // ... + barriers + TMEM slot and flags + cpre[E + 1] + soff[E + 1]
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STAGE_OUT_BYTES + SA_BYTES +
-                                    NUM_BARS * 8 + 16 + (MAX_E + 8) * 4;
+                                    NUM_BARS * 8 + 16 + 2 * (MAX_E + 8) * 4;
   static_assert(TMEM_COLS <= 512 && (TMEM_COLS & (TMEM_COLS - 1)) == 0, "tensor memory");
   static_assert(!kFp8 || TN <= 64, "FP8 keeps TN columns per K-block buffer, 4 buffers");
   static constexpr int WROWS = (kMode == kTSwiglu) ? 64 : 128;  // output columns per tile
@@ -103,25 +108,20 @@ struct TTile {
 };
 
 // Tile t -> (expert, weight block, token chunk). cpre[e] = token chunks of the
-// experts before e (shared memory, built at kernel start); WB weight blocks.
-__device__ __forceinline__ bool t_decode(const TParams& p, const int* cpre, int E, int WB, int TN,
-                                         int t, TTile& ti) {
-  int lo = 0, hi = E - 1;  // largest e with WB*cpre[e] <= t
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (WB * cpre[mid] <= t)
-      lo = mid;
-    else
-      hi = mid - 1;
-  }
-  const int e = lo;
+// experts before e and soff[e] = group_offsets[e] (both in shared memory, built
+// at kernel start); WB weight blocks. A CTA visits its tiles in increasing
+// order, so each warp keeps the expert of its last tile in `ecur` and only
+// moves it forward: no search and no global load per tile.
+__device__ __forceinline__ bool t_decode(const TParams& p, const int* cpre, const int* soff,
+                                         int WB, int TN, int t, int& ecur, TTile& ti) {
+  while (WB * cpre[ecur + 1] <= t) ++ecur;  // experts without chunks are passed over
+  const int e = ecur;
   const int chunks = cpre[e + 1] - cpre[e];
-  if (chunks <= 0) return false;
   const int local = t - WB * cpre[e];
   const int wb = local / chunks;
   const int c = local - wb * chunks;
-  const int size = p.group_sizes ? __ldg(p.group_sizes + e) : p.M_dense;
-  const int off = p.group_offsets ? __ldg(p.group_offsets + e) : 0;
+  const int off = soff[e];
+  const int size = soff[e + 1] - off;
   ti.e = e;
   ti.wb = wb;
   ti.chunks = chunks;
@@ -210,7 +210,7 @@ __device__ __forceinline__ void store_rows(const TParams& p, const float* sOut, 
 }
 
 template <int kMode, int TN>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(TCfg<kMode, TN>::kThreads, 1)
     grouped_gemm_t_kernel(const __grid_constant__ CUtensorMap tmW,
                           const __grid_constant__ CUtensorMap tmX0,
                           const __grid_constant__ CUtensorMap tmX1,
@@ -228,7 +228,8 @@ __global__ void __launch_bounds__(192, 1)
   float* sOut = reinterpret_cast<float*>(sB + STAGES * Cfg::B_BYTES);  // [32][128]
   int* sDst = reinterpret_cast<int*>(sOut + 32 * 128);  // weighted store: the tile's row info
   float* sFac = reinterpret_cast<float*>(sDst + TN);
-  float* sSa = sOut + 32 * 128 + 2 * TN;  // FP8: activation scales of the tile's tokens [TN][KBS]
+  // FP8: sa * sw of a tile's tokens, K-block major [KBS][TN], two slots
+  float* sSa = sOut + 32 * 128 + 2 * TN;
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sOut) +
                                                Cfg::STAGE_OUT_BYTES + Cfg::SA_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NUM_BARS);
@@ -237,12 +238,16 @@ __global__ void __launch_bounds__(192, 1)
   // epilogue warps always agree on whether to stop
   volatile int* epi_abort = reinterpret_cast<volatile int*>(tmem_slot + 2);
   int* cpre = reinterpret_cast<int*>(tmem_slot + 4);  // [E + 1]
+  int* soff = cpre + Cfg::MAX_E + 8;                    // [E + 1]: group_offsets
 
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = full0 + 8 * STAGES;
   const uint32_t tfull0 = empty0 + 8 * STAGES;
   const uint32_t tempty0 = tfull0 + 8 * NUM_ACC;
   const uint32_t drain_bar = tempty0 + 8 * NUM_ACC;
+  const uint32_t scl_full0 = drain_bar + 8;      // FP8: slot filled by the scale warp
+  const uint32_t scl_empty0 = scl_full0 + 16;    // FP8: slot released by the epilogue
+  constexpr int kThreads = Cfg::kThreads;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -258,6 +263,12 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(tempty0 + 8 * a, 4);
     }
     mbar_init(drain_bar, 1);
+    if constexpr (Cfg::kFp8) {
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(scl_full0 + 8 * i, 1);
+        mbar_init(scl_empty0 + 8 * i, 1);
+      }
+    }
     *abort_flag = 0;
     *epi_abort = 0;
     mbar_fence_init();
@@ -270,9 +281,9 @@ __global__ void __launch_bounds__(192, 1)
     tma_prefetch_desc(&tmX3);
   }
   if (warp == 1) tmem_alloc(smem_u32(tmem_slot), Cfg::TMEM_COLS);
-  // token chunks per expert -> exclusive prefix cpre[0..E] (192 threads)
+  // token chunks per expert -> exclusive prefix cpre[0..E] (all threads)
   {
-    const int per = (E + 191) / 192;
+    const int per = (E + kThreads - 1) / kThreads;
     const int beg = threadIdx.x * per;
     int local = 0;
     for (int i = 0; i < per && beg + i < E; ++i) {
@@ -296,7 +307,9 @@ __global__ void __launch_bounds__(192, 1)
       const int s = p.group_sizes ? __ldg(p.group_sizes + beg + i) : p.M_dense;
       run += (s + TN - 1) / TN;
     }
-    if (threadIdx.x == 191) cpre[E] = before + inc;
+    if (threadIdx.x == kThreads - 1) cpre[E] = before + inc;
+    for (int i = threadIdx.x; i <= E; i += kThreads)
+      soff[i] = p.group_offsets ? __ldg(p.group_offsets + i) : (i == 0 ? 0 : p.M_dense);
   }
   tc_fence_before();
   __syncthreads();
@@ -318,9 +331,10 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t phase = 0;
       uint32_t issued = 0;
       bool ok = true;
+      int ecur = 0;
       for (int t = blockIdx.x; ok && t < total_tiles; t += gridDim.x) {
         TTile ti;
-        if (!t_decode(p, cpre, E, WB, TN, t, ti)) continue;
+        if (!t_decode(p, cpre, soff, WB, TN, t, ecur, ti)) continue;
         const int nmma = (ti.nt + 15) & ~15;
         const int xb = xbox_for(nmma);
         const uint32_t bytes = Cfg::A_BYTES + (32u << xb) * 128u;
@@ -370,9 +384,10 @@ __global__ void __launch_bounds__(192, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
+      int ecur = 0;
       for (int t = blockIdx.x; ok && t < total_tiles; t += gridDim.x) {
         TTile ti;
-        if (!t_decode(p, cpre, E, WB, TN, t, ti)) continue;
+        if (!t_decode(p, cpre, soff, WB, TN, t, ecur, ti)) continue;
         const int nmma = (ti.nt + 15) & ~15;
         if constexpr (Cfg::kFp8) {
           // one TMEM buffer per 128-wide K-block: the epilogue scales and sums them
@@ -438,6 +453,55 @@ __global__ void __launch_bounds__(192, 1)
       mma_commit(drain_bar);
       mbar_wait_drain(drain_bar, 0);
     }
+  } else if (warp == 6) {
+    // ------------------------------------------------------------ scale warp (FP8)
+    // For each tile, one tile ahead of the epilogue: s[kb][t] = sw[e, wb, kb] *
+    // sa[m0 + t, kb] into the next slot of the two-slot ring, K-block major so
+    // the epilogue reads each K-block's column scales as 16-byte broadcasts. It
+    // keeps the global loads' latency off the epilogue's path.
+    if constexpr (Cfg::kFp8) {
+      int ecur = 0;
+      int slot = 0;
+      uint32_t sphase = 0;
+      for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+        TTile ti;
+        if (!t_decode(p, cpre, soff, WB, TN, t, ecur, ti)) continue;
+        uint32_t got = 1;
+        if (lane == 0) got = mbar_wait(scl_empty0 + 8 * slot, sphase ^ 1u, abort_flag, p.status);
+        if (!__shfl_sync(0xffffffffu, got, 0)) break;
+        float* dst = sSa + slot * Cfg::SA_SLOT;
+        const int nsa = ti.nt * p.KBS;
+        const float* gsa = p.A_scales + static_cast<int64_t>(ti.m0) * p.KBS;
+        const float* gsw =
+            p.B_scales + (static_cast<int64_t>(ti.e) * (p.N / 128) + ti.wb) * p.KBS;
+        // 8 independent loads in flight per lane per round (at most 4 rounds)
+        for (int base = 0; base < nsa; base += 8 * 32) {
+          float a[8], b[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int i = base + j * 32 + lane;
+            const bool in = i < nsa;
+            a[j] = in ? __ldg(gsa + i) : 0.0f;
+            b[j] = in ? __ldg(gsw + (i % p.KBS)) : 0.0f;
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int i = base + j * 32 + lane;
+            if (i < nsa) {
+              const int tok = i / p.KBS;
+              const int kb = i - tok * p.KBS;
+              dst[kb * TN + tok] = a[j] * b[j];
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(scl_full0 + 8 * slot);
+        if (++slot == 2) {
+          slot = 0;
+          sphase ^= 1u;
+        }
+      }
+    }
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
@@ -447,40 +511,20 @@ __global__ void __launch_bounds__(192, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     int stage = 0;  // FP8: the shared-memory stage of the next K-block, as the MMA thread counts
+    int sslot = 0;  // FP8: the scale ring's slot of the next tile, and its phase
+    uint32_t sphase = 0;
+    int ecur = 0;
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
       TTile ti;
-      if (!t_decode(p, cpre, E, WB, TN, t, ti)) continue;
+      if (!t_decode(p, cpre, soff, WB, TN, t, ecur, ti)) continue;
       if (kMode != kTSwiglu && p.weighted) stage_row_info(p, et, ti.nt, ti.m0, sDst, sFac);
       if constexpr (Cfg::kFp8) {
-        // y[t, w] = sum_kb sw[e, wb, kb] * sa[t, kb] * (Wq_kb Xq_kb^T)[w, t]
-        // stage s[kb][t] = sw[e, wb, kb] * sa[m0 + t, kb], K-block major so each
-        // K-block's column scales are read as 16-byte vectors (same address in
-        // every thread: a broadcast)
-        const int nsa = ti.nt * p.KBS;
-        const float* gsa = p.A_scales + static_cast<int64_t>(ti.m0) * p.KBS;
-        const float* gsw =
-            p.B_scales + (static_cast<int64_t>(ti.e) * (p.N / 128) + ti.wb) * p.KBS;
-        // 8 independent loads in flight per thread per round (at most TN*32/1024 rounds)
-        for (int base = 0; base < nsa; base += 8 * 128) {
-          float a[8], b[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int i = base + j * 128 + et;
-            const bool in = i < nsa;
-            a[j] = in ? __ldg(gsa + i) : 0.0f;
-            b[j] = in ? __ldg(gsw + (i % p.KBS)) : 0.0f;
-          }
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int i = base + j * 128 + et;
-            if (i < nsa) {
-              const int tok = i / p.KBS;
-              const int kb = i - tok * p.KBS;
-              sSa[kb * TN + tok] = a[j] * b[j];
-            }
-          }
-        }
-        epi_bar();
+        // y[t, w] = sum_kb sw[e, wb, kb] * sa[t, kb] * (Wq_kb Xq_kb^T)[w, t], with
+        // the tile's products sw * sa prepared by the scale warp in slot sslot
+        const float* sS = sSa + sslot * Cfg::SA_SLOT;
+        if (!mbar_wait(scl_full0 + 8 * sslot, sphase, abort_flag, p.status)) *epi_abort = 1;
+        epi_bar();  // every epilogue warp arrives here whether its wait succeeded or not
+        if (*epi_abort) break;
         float accv[TN];
 #pragma unroll
         for (int i = 0; i < TN; ++i) accv[i] = 0.0f;
@@ -495,7 +539,7 @@ __global__ void __launch_bounds__(192, 1)
           if (++stage == STAGES) stage = 0;
           tc_fence_after();
           const uint32_t tbk = lane_base + static_cast<uint32_t>(acc * TN);
-          const float4* s4 = reinterpret_cast<const float4*>(sSa + kb * TN);
+          const float4* s4 = reinterpret_cast<const float4*>(sS + kb * TN);
           uint32_t v[TN / 32][32];
 #pragma unroll
           for (int c = 0; c < TN / 32; ++c)
@@ -526,6 +570,12 @@ __global__ void __launch_bounds__(192, 1)
         if (!ok) *epi_abort = 1;
         epi_bar();
         if (*epi_abort) break;
+        // every epilogue thread is done with the slot: the scale warp may refill it
+        if (et == 0) mbar_arrive(scl_empty0 + 8 * sslot);
+        if (++sslot == 2) {
+          sslot = 0;
+          sphase ^= 1u;
+        }
 #pragma unroll
         for (int c = 0; c < TN / 32; ++c) {
           if (c * 32 < ti.nt) {
@@ -683,7 +733,7 @@ cudaError_t run_t(const GemmLaunch& L, cudaStream_t stream) {
   const long long tiles_ub = chunks_ub * WB;
   const int sms = device_sm_count();
   const int grid = static_cast<int>(tiles_ub < sms ? (tiles_ub > 0 ? tiles_ub : 1) : sms);
-  grouped_gemm_t_kernel<kMode, TN><<<grid, 192, Cfg::SMEM_BYTES, stream>>>(
+  grouped_gemm_t_kernel<kMode, TN><<<grid, Cfg::kThreads, Cfg::SMEM_BYTES, stream>>>(
       tmW, tmX[0], tmX[1], tmX[2], tmX[3], p);
   return cudaGetLastError();
 }
@@ -698,7 +748,7 @@ bool grouped_gemm_t_supported(const GemmLaunch& L) {
     return false;
   if (L.mode == kModeFp8Store)
     return L.A_scales != nullptr && L.B_scales != nullptr && L.N % 128 == 0 &&
-           L.K % 128 == 0 && L.K <= 128 * 32;
+           L.K % 128 == 0 && L.K <= 128 * TCfg<kTFp8Store, 64>::MAX_KBS;
   if (L.A_scales != nullptr || L.B_scales != nullptr) return false;
   if (L.mode == kModeStore) return L.N % 128 == 0 && L.K % 64 == 0;
   if (L.mode == kModeSwiglu) return (L.N / 2) % 64 == 0 && L.N % 2 == 0 && L.K % 64 == 0;

@@ -30,7 +30,6 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
-#include <algorithm>
 #include <mutex>
 
 #include "internal.h"
@@ -70,18 +69,6 @@ struct PParams {
 
 __host__ __device__ constexpr int pmin(int a, int b) { return a < b ? a : b; }
 
-// Kernel arguments: up to two independent problems of the same mode and token
-// tile. Pairs [0, pairs_b) compute problem 1, the other pairs problem 0 (a
-// launch with one problem has pairs_b == 0). Two problems in one launch let
-// a compute-bound dense problem (the shared expert) run on a few SM pairs
-// while the memory-bound routed experts stream their weights on the rest.
-struct PairArgs {
-  CUtensorMap w[2];             // weights of problem 0 / 1
-  CUtensorMap x[2][kPXBoxes];   // token rows: boxes of 16, 32, 64, 128 rows
-  PParams p[2];
-  int pairs_b;
-};
-
 template <int kMode, int TN>
 struct PCfg {
   static constexpr int BK = 64;
@@ -98,7 +85,7 @@ struct PCfg {
   static constexpr int NUM_BARS = 2 * STAGES + 2 * NUM_ACC + 1;
   static constexpr int MAX_E = 1024;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STAGE_OUT_BYTES +
-                                    NUM_BARS * 8 + 16 + (MAX_E + 8) * 4;
+                                    NUM_BARS * 8 + 16 + 2 * (MAX_E + 8) * 4;
   static constexpr int PAIR_COLS = (kMode == kPSwiglu) ? 128 : 256;  // output columns per pair tile
   static constexpr int CTA_COLS = PAIR_COLS / 2;
   static_assert(TN % 32 == 0 && TN >= 32 && TN <= 256, "token tile");
@@ -111,24 +98,20 @@ struct PTile {
   int chunks;  // token tiles of this expert (tiles that read the same weights)
 };
 
-__device__ __forceinline__ bool p_decode(const PParams& p, const int* cpre, int E, int WB, int TN,
-                                         int t, PTile& ti) {
-  int lo = 0, hi = E - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (WB * cpre[mid] <= t)
-      lo = mid;
-    else
-      hi = mid - 1;
-  }
-  const int e = lo;
+// Tile t -> (expert, weight block, token chunk), from cpre (token chunks of the
+// experts before e) and soff (group_offsets), both in shared memory. A pair
+// visits its tiles in increasing order, so each warp keeps the expert of its
+// last tile in `ecur` and only moves it forward.
+__device__ __forceinline__ bool p_decode(const PParams& p, const int* cpre, const int* soff,
+                                         int WB, int TN, int t, int& ecur, PTile& ti) {
+  while (WB * cpre[ecur + 1] <= t) ++ecur;  // experts without chunks are passed over
+  const int e = ecur;
   const int chunks = cpre[e + 1] - cpre[e];
-  if (chunks <= 0) return false;
   const int local = t - WB * cpre[e];
   const int wb = local / chunks;
   const int c = local - wb * chunks;
-  const int size = p.group_sizes ? __ldg(p.group_sizes + e) : p.M_dense;
-  const int off = p.group_offsets ? __ldg(p.group_offsets + e) : 0;
+  const int off = soff[e];
+  const int size = soff[e + 1] - off;
   ti.e = e;
   ti.wb = wb;
   ti.chunks = chunks;
@@ -162,7 +145,11 @@ constexpr int kPairThreads = 192;
 
 template <int kMode, int TN, bool kGather>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
-    grouped_gemm_pair_kernel(const __grid_constant__ PairArgs args) {
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmW,
+                             const __grid_constant__ CUtensorMap tmX0,
+                             const __grid_constant__ CUtensorMap tmX1,
+                             const __grid_constant__ CUtensorMap tmX2,
+                             const __grid_constant__ CUtensorMap tmX3, const PParams p) {
   using Cfg = PCfg<kMode, TN>;
   constexpr int STAGES = Cfg::STAGES;
   constexpr int NUM_ACC = Cfg::NUM_ACC;
@@ -181,7 +168,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NUM_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* epi_abort = reinterpret_cast<volatile int*>(tmem_slot + 2);
-  int* cpre = reinterpret_cast<int*>(tmem_slot + 4);
+  int* cpre = reinterpret_cast<int*>(tmem_slot + 4);  // [E + 1]
+  int* soff = cpre + Cfg::MAX_E + 8;                    // [E + 1]: group_offsets
 
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = full0 + 8 * STAGES;
@@ -191,17 +179,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int E = p.group_sizes ? p.E : 1;
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
-  // this pair's problem, and its index among the pairs of that problem
-  const int pair_all = blockIdx.x >> 1;
-  const int role = pair_all < args.pairs_b ? 1 : 0;
-  const PParams& p = args.p[role];
-  const CUtensorMap* tmW = &args.w[role];
-  const CUtensorMap* tmX = args.x[role];
-  const int pair = role ? pair_all : pair_all - args.pairs_b;
-  const int npairs = role ? args.pairs_b : (gridDim.x >> 1) - args.pairs_b;
-  const int E = p.group_sizes ? p.E : 1;
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -218,8 +200,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     mbar_fence_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(tmW);
-    for (int i = 0; i < kPXBoxes; ++i) tma_prefetch_desc(&tmX[i]);
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmX0);
+    tma_prefetch_desc(&tmX1);
+    tma_prefetch_desc(&tmX2);
+    tma_prefetch_desc(&tmX3);
   }
   if (warp == 1) tmem_alloc_pair(smem_u32(tmem_slot), Cfg::TMEM_COLS);
   {
@@ -248,6 +233,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       run += (s + TN - 1) / TN;
     }
     if (threadIdx.x == kThreads - 1) cpre[E] = before + inc;
+    for (int i = threadIdx.x; i <= E; i += kThreads)
+      soff[i] = p.group_offsets ? __ldg(p.group_offsets + i) : (i == 0 ? 0 : p.M_dense);
   }
   tc_fence_before();
   __syncthreads();
@@ -270,13 +257,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       const uint64_t pol_act = l2_policy_evict_last();
       const uint64_t pol_w1 = l2_policy_by_code(MOE_W_POLICY_SINGLE);
       const uint64_t pol_wn = l2_policy_by_code(MOE_W_POLICY_MULTI);
+      const CUtensorMap* xmaps[kPXBoxes] = {&tmX0, &tmX1, &tmX2, &tmX3};
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued = 0;  // stages whose loads this CTA issued
       bool ok = true;
+      int ecur = 0;
       for (int t = pair; ok && t < total_tiles; t += npairs) {
         PTile ti;
-        if (!p_decode(p, cpre, E, WB, TN, t, ti)) continue;
+        if (!p_decode(p, cpre, soff, WB, TN, t, ecur, ti)) continue;
         const int nmma = (ti.nt + 31) & ~31;
         const int half = nmma / 2;
         const int xb = half_box(half);
@@ -317,16 +306,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             if (leader) mbar_arrive_expect_tx(fb_local, bytes_pair);
             const uint32_t a_dst = smem_u32(sA + stage * Cfg::A_BYTES);
             if constexpr (kMode == kPSwiglu) {
-              tma_load_2d_pair(a_dst, tmW, kb * Cfg::BK, wrow, fb, pol_w);
-              tma_load_2d_pair(a_dst + 64 * 128, tmW, kb * Cfg::BK, wrow + p.up_off, fb, pol_w);
+              tma_load_2d_pair(a_dst, &tmW, kb * Cfg::BK, wrow, fb, pol_w);
+              tma_load_2d_pair(a_dst + 64 * 128, &tmW, kb * Cfg::BK, wrow + p.up_off, fb, pol_w);
             } else {
-              tma_load_2d_pair(a_dst, tmW, kb * Cfg::BK, wrow, fb, pol_w);
+              tma_load_2d_pair(a_dst, &tmW, kb * Cfg::BK, wrow, fb, pol_w);
             }
             if constexpr (!kGather)
-              tma_load_2d_pair(b_dst, &tmX[xb], kb * Cfg::BK, trow, fb, pol_act);
+              tma_load_2d_pair(b_dst, xmaps[xb], kb * Cfg::BK, trow, fb, pol_act);
           }
           if (gather_lane)
-            tma_gather4_pair(b_dst + lane * 512, &tmX[0], kb * Cfg::BK, g[0], g[1], g[2], g[3], fb,
+            tma_gather4_pair(b_dst + lane * 512, &tmX0, kb * Cfg::BK, g[0], g[1], g[2], g[3], fb,
                              pol_act);
           ++issued;
           if (++stage == STAGES) {
@@ -379,9 +368,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
+      int ecur = 0;
       for (int t = pair; ok && t < total_tiles; t += npairs) {
         PTile ti;
-        if (!p_decode(p, cpre, E, WB, TN, t, ti)) continue;
+        if (!p_decode(p, cpre, soff, WB, TN, t, ecur, ti)) continue;
         const int nmma = (ti.nt + 31) & ~31;
         const uint32_t idesc = idesc_bf16_f32(256, nmma);
         if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag, p.status)) {
@@ -425,9 +415,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     int acc = 0;
     uint32_t acc_phase = 0;
+    int ecur = 0;
     for (int t = pair; t < total_tiles; t += npairs) {
       PTile ti;
-      if (!p_decode(p, cpre, E, WB, TN, t, ti)) continue;
+      if (!p_decode(p, cpre, soff, WB, TN, t, ecur, ti)) continue;
       if (kMode == kPStore && p.weighted) {
         // the tile's row destinations (flat pair index, -1 = none) and factors,
         // loaded while its MMAs run; read after the first chunk's barrier
@@ -572,63 +563,43 @@ bool p_encode(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows, uin
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Pairs of the kernel instantiation that can be resident at once (a pair needs
-// both SMs of one TPC free); sets the kernel's shared-memory attribute on first
-// use. 0 on error (*err set).
 template <int kMode, int TN, bool kGather>
-int pair_capacity(cudaError_t* err) {
+cudaError_t run_pair(const GemmLaunch& L, cudaStream_t stream) {
   using Cfg = PCfg<kMode, TN>;
+  constexpr int kThreads = kPairThreads;
   static int max_pairs_cache[64] = {0};
   int dev = 0;
-  *err = cudaGetDevice(&dev);
-  if (*err != cudaSuccess) return 0;
-  if (dev < 0 || dev >= 64) {
-    *err = cudaErrorInvalidDevice;
-    return 0;
-  }
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (max_pairs_cache[dev] == 0) {
-    *err = cudaFuncSetAttribute(grouped_gemm_pair_kernel<kMode, TN, kGather>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
-    if (*err != cudaSuccess) return 0;
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_pair_kernel<kMode, TN, kGather>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Cfg::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    // pairs that can be resident at once (a pair needs both SMs of one TPC free)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(device_sm_count() & ~1));
-    cfg.blockDim = dim3(kPairThreads);
+    cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
     int n = 0;
-    *err = cudaOccupancyMaxActiveClusters(&n, grouped_gemm_pair_kernel<kMode, TN, kGather>, &cfg);
-    if (*err != cudaSuccess) return 0;
+    e = cudaOccupancyMaxActiveClusters(&n, grouped_gemm_pair_kernel<kMode, TN, kGather>, &cfg);
+    if (e != cudaSuccess) return e;
     max_pairs_cache[dev] = n > 0 ? n : 1;
   }
-  *err = cudaSuccess;
-  return max_pairs_cache[dev];
-}
-
-// Upper bound of the pair tiles of a problem (token chunks x weight blocks).
-template <int kMode, int TN>
-long long pair_tiles_ub(const GemmLaunch& L) {
-  const bool grouped = L.group_sizes != nullptr;
-  const int WB = kMode == kPSwiglu ? (L.N / 2) / 128 : L.N / 256;
-  const long long chunks_ub = grouped ? (static_cast<long long>(L.rows) + TN - 1) / TN + L.E
-                                      : (static_cast<long long>(L.rows) + TN - 1) / TN;
-  return chunks_ub * WB;
-}
-
-// Tensor maps and parameters of problem `slot` of the argument block.
-template <int kMode, int TN, bool kGather>
-bool fill_pair_problem(const GemmLaunch& L, PairArgs& a, int slot) {
   const bool grouped = L.group_sizes != nullptr;
   const int E = grouped ? L.E : 1;
   // rows of the A operand in memory: the hidden states in gather mode
   const int a_rows = kGather ? L.a_rows : L.rows;
+  CUtensorMap tmW, tmX[kPXBoxes];
   const uint64_t b_rows = L.b_rows > 0 ? static_cast<uint64_t>(L.b_rows) : static_cast<uint64_t>(E) * L.N;
   const uint64_t ldb = L.ldb > 0 ? static_cast<uint64_t>(L.ldb) : static_cast<uint64_t>(L.K);
-  if (!p_encode(&a.w[slot], L.B, L.K, b_rows, kMode == kPSwiglu ? 64 : 128, ldb)) return false;
+  if (!p_encode(&tmW, L.B, L.K, b_rows, kMode == kPSwiglu ? 64 : 128, ldb))
+    return cudaErrorInvalidValue;
   // gather mode: map 0 is the hidden states with a one-row-high box (four-row gathers)
   for (int i = 0; i < kPXBoxes; ++i)
-    if (!p_encode(&a.x[slot][i], L.A, L.K, a_rows, kGather && i == 0 ? 1u : 16u << i, L.K))
-      return false;
-  PParams& p = a.p[slot];
-  p = PParams{};
+    if (!p_encode(&tmX[i], L.A, L.K, a_rows, kGather && i == 0 ? 1u : 16u << i, L.K))
+      return cudaErrorInvalidValue;
+  PParams p{};
   p.M_dense = grouped ? 0 : L.rows;
   p.N = L.N;
   p.K = L.K;
@@ -648,106 +619,20 @@ bool fill_pair_problem(const GemmLaunch& L, PairArgs& a, int slot) {
   p.weighted = L.weighted;
   p.row_w = L.row_weights;
   p.row_scale = L.row_scale;
-  return true;
-}
-
-// One problem (L1 == nullptr, pairs_b ignored) on as many pairs as it has
-// tiles, up to the resident maximum; or two problems on all resident pairs,
-// pairs_b of them (1 .. max - 1) on L1.
-template <int kMode, int TN, bool kGather>
-cudaError_t run_pair(const GemmLaunch& L0, const GemmLaunch* L1, int pairs_b,
-                     cudaStream_t stream) {
-  using Cfg = PCfg<kMode, TN>;
-  cudaError_t e = cudaSuccess;
-  const int max_pairs = pair_capacity<kMode, TN, kGather>(&e);
-  if (max_pairs == 0) return e;
-  PairArgs a;
-  if (!fill_pair_problem<kMode, TN, kGather>(L0, a, 0)) return cudaErrorInvalidValue;
-  int pairs = 0;
-  if (L1 == nullptr) {
-    a.w[1] = a.w[0];
-    for (int i = 0; i < kPXBoxes; ++i) a.x[1][i] = a.x[0][i];
-    a.p[1] = a.p[0];
-    a.pairs_b = 0;
-    const long long ub = pair_tiles_ub<kMode, TN>(L0);
-    pairs = static_cast<int>(ub < max_pairs ? (ub > 0 ? ub : 1) : max_pairs);
-  } else {
-    if (pairs_b < 1 || pairs_b >= max_pairs) return cudaErrorInvalidValue;
-    if (!fill_pair_problem<kMode, TN, kGather>(*L1, a, 1)) return cudaErrorInvalidValue;
-    a.pairs_b = pairs_b;
-    pairs = max_pairs;
-  }
-  grouped_gemm_pair_kernel<kMode, TN, kGather><<<2 * pairs, kPairThreads, Cfg::SMEM_BYTES, stream>>>(a);
+  const int WB = kMode == kPSwiglu ? (L.N / 2) / 128 : L.N / 256;
+  const long long chunks_ub = grouped ? (static_cast<long long>(L.rows) + TN - 1) / TN + E
+                                      : (static_cast<long long>(L.rows) + TN - 1) / TN;
+  const long long pairs_ub = chunks_ub * WB;
+  const int max_pairs = max_pairs_cache[dev];
+  const int pairs = static_cast<int>(pairs_ub < max_pairs ? (pairs_ub > 0 ? pairs_ub : 1) : max_pairs);
+  grouped_gemm_pair_kernel<kMode, TN, kGather><<<2 * pairs, kThreads, Cfg::SMEM_BYTES, stream>>>(
+      tmW, tmX[0], tmX[1], tmX[2], tmX[3], p);
   return cudaGetLastError();
 }
 
 template <int kMode, int TN>
 cudaError_t run_pair_g(const GemmLaunch& L, cudaStream_t stream) {
-  return L.gather ? run_pair<kMode, TN, true>(L, nullptr, 0, stream)
-                  : run_pair<kMode, TN, false>(L, nullptr, 0, stream);
-}
-
-// Token tile of the pair kernel for a problem: 64 for small groups (decode);
-// 128 for a dense problem too small to give three quarters of the CTA pairs a
-// 256-token tile (a tensor-parallel rank's shared expert, few tokens: twice
-// the tiles, and the MMA still runs at its full rate from N = 128; one rank of
-// tp 8 at Kimi-K2's shared expert: 36 -> 72 tiles); else 256.
-int pair_token_tile(const GemmLaunch& L) {
-  const bool small = L.group_sizes != nullptr && L.rows <= 64 * L.E;
-  if (small) return 64;
-  if (L.group_sizes == nullptr && L.rows > 128) {
-    const long long wb = L.mode == kModeSwiglu ? (L.N / 2) / 128 : L.N / 256;
-    const long long tiles256 = wb * ((static_cast<long long>(L.rows) + 255) / 256);
-    if (tiles256 * 4 < static_cast<long long>(device_sm_count() / 2) * 3) return 128;
-  }
-  return 256;
-}
-
-// Split of the resident pairs between a memory-bound problem L0 and a
-// compute-bound problem L1 sharing one launch: the smallest share for L1 whose
-// estimated time (its FLOPs at a conservative per-pair MMA rate) does not
-// exceed L0's (the larger of its weight and output bytes at a conservative HBM
-// rate and its FLOPs on the remaining pairs). 0 when sharing is not estimated
-// to beat two launches one after the other.
-int pair_dual_split(const GemmLaunch& L0, const GemmLaunch& L1, int max_pairs) {
-  if (max_pairs < 4) return 0;
-  constexpr double kPairFlops = 2.0e13;  // FLOP/s of one CTA pair (power-capped clocks)
-  constexpr double kHbm = 6.0e12;        // B/s
-  auto flops = [](const GemmLaunch& L) { return 2.0 * L.rows * static_cast<double>(L.N) * L.K; };
-  auto bytes = [](const GemmLaunch& L) {
-    const double w = static_cast<double>(L.group_sizes ? L.E : 1) * L.N * L.K * 2.0;
-    const double out = L.mode == kModeSwiglu ? L.rows * (L.N / 2) * 2.0
-                                             : L.rows * static_cast<double>(L.N) * (L.out_f32 ? 4 : 2);
-    return w + out;
-  };
-  const double t0_mem = bytes(L0) / kHbm;
-  const double t1_mem = bytes(L1) / kHbm;
-  const double seq = std::max(t0_mem, flops(L0) / (max_pairs * kPairFlops)) +
-                     std::max(t1_mem, flops(L1) / (max_pairs * kPairFlops));
-  int best = 0;
-  double best_t = seq;
-  for (int pb = 1; pb < max_pairs; ++pb) {
-    const double t0 = std::max(t0_mem, flops(L0) / ((max_pairs - pb) * kPairFlops));
-    const double t1 = flops(L1) / (pb * kPairFlops);
-    const double t = std::max(t0, t1);
-    if (t < best_t * 0.97) {
-      best_t = t;
-      best = pb;
-    }
-  }
-  return best;
-}
-
-template <int kMode, int TN>
-cudaError_t run_pair_dual(const GemmLaunch& L0, const GemmLaunch& L1, cudaStream_t stream,
-                          bool* done) {
-  cudaError_t e = cudaSuccess;
-  const int max_pairs = pair_capacity<kMode, TN, false>(&e);
-  if (max_pairs == 0) return e;
-  const int pb = pair_dual_split(L0, L1, max_pairs);
-  if (pb == 0) return cudaSuccess;   // *done stays false: the caller launches both
-  *done = true;
-  return run_pair<kMode, TN, false>(L0, &L1, pb, stream);
+  return L.gather ? run_pair<kMode, TN, true>(L, stream) : run_pair<kMode, TN, false>(L, stream);
 }
 
 }  // namespace
@@ -779,30 +664,26 @@ bool grouped_gemm_pair_preferred(const GemmLaunch& L) {
 }
 
 cudaError_t launch_grouped_gemm_pair(const GemmLaunch& L, cudaStream_t stream) {
-  const int tn = pair_token_tile(L);
+  const bool small = L.group_sizes != nullptr && L.rows <= 64 * L.E;
+  // A dense problem too small to give three quarters of the CTA pairs a
+  // 256-token tile (a tensor-parallel rank's shared expert, few tokens) takes
+  // 128-token tiles: twice the tiles, and the MMA still runs at its full rate
+  // from N = 128 (one rank of tp 8 at Kimi-K2's shared expert: 36 -> 72 tiles).
+  bool mid = false;
+  if (!small && L.group_sizes == nullptr && L.rows > 128) {
+    const long long wb = L.mode == kModeSwiglu ? (L.N / 2) / 128 : L.N / 256;
+    const long long tiles256 = wb * ((static_cast<long long>(L.rows) + 255) / 256);
+    mid = tiles256 * 4 < static_cast<long long>(device_sm_count() / 2) * 3;
+  }
   if (L.mode == kModeSwiglu)
-    return tn == 64 ? run_pair_g<kPSwiglu, 64>(L, stream)
-                    : tn == 128 ? run_pair_g<kPSwiglu, 128>(L, stream)
-                                : run_pair_g<kPSwiglu, 256>(L, stream);
+    return small ? run_pair_g<kPSwiglu, 64>(L, stream)
+                 : mid ? run_pair_g<kPSwiglu, 128>(L, stream)
+                       : run_pair_g<kPSwiglu, 256>(L, stream);
   if (L.mode == kModeStore)
-    return tn == 64 ? run_pair_g<kPStore, 64>(L, stream)
-                    : tn == 128 ? run_pair_g<kPStore, 128>(L, stream)
-                                : run_pair_g<kPStore, 256>(L, stream);
+    return small ? run_pair_g<kPStore, 64>(L, stream)
+                 : mid ? run_pair_g<kPStore, 128>(L, stream)
+                       : run_pair_g<kPStore, 256>(L, stream);
   return cudaErrorInvalidValue;
-}
-
-cudaError_t launch_grouped_gemm_pair_dual(const GemmLaunch& L0, const GemmLaunch& L1,
-                                          cudaStream_t stream, bool* done) {
-  *done = false;
-  if (!grouped_gemm_pair_preferred(L0) || !grouped_gemm_pair_preferred(L1)) return cudaSuccess;
-  if (L0.gather || L1.gather || L0.mode != L1.mode || L1.group_sizes != nullptr ||
-      L0.weighted || L1.weighted)
-    return cudaSuccess;
-  const int tn = pair_token_tile(L0);
-  if (tn != 256 || pair_token_tile(L1) != 256) return cudaSuccess;
-  if (L0.mode == kModeSwiglu) return run_pair_dual<kPSwiglu, 256>(L0, L1, stream, done);
-  if (L0.mode == kModeStore) return run_pair_dual<kPStore, 256>(L0, L1, stream, done);
-  return cudaSuccess;
 }
 
 }  // namespace moe

@@ -68,13 +68,6 @@ bool grouped_gemm_t_preferred(const GemmLaunch& L);
 cudaError_t launch_grouped_gemm_pair(const GemmLaunch& L, cudaStream_t stream);
 bool grouped_gemm_pair_supported(const GemmLaunch& L);
 bool grouped_gemm_pair_preferred(const GemmLaunch& L);
-// Two problems in one launch of the pair kernel: L0 (memory-bound: the routed
-// experts) on most of the resident pairs and the dense L1 (compute-bound: the
-// shared expert) on a few, when both take the same kernel instantiation and
-// the split is estimated to beat two launches. *done = false (and nothing
-// launched) otherwise.
-cudaError_t launch_grouped_gemm_pair_dual(const GemmLaunch& L0, const GemmLaunch& L1,
-                                          cudaStream_t stream, bool* done);
 
 cudaError_t launch_route_topk(const float* logits, int T, int E, int k, int score_fn,
                               int renormalize, int32_t* ids, float* weights, cudaStream_t stream);

@@ -186,34 +186,6 @@ def test_deterministic_repeat():
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
-def test_shared_expert_in_the_routed_launch():
-    """A workload whose routed gate+up GEMM is weight-bound and whose shared
-    expert is compute-bound: the shared gate+up runs in the same pair-kernel
-    launch as the routed one, on pairs of its own (one launch fewer), and every
-    output element matches the oracle."""
-    import moe_routed_expert_top_b200 as M
-    gu = _gu()
-    cfg = get_config("tiny", name="shared_dual", T=1024, E=16, top_k=2, H=2048, F=1024,
-                     score_fn="sigmoid", routed_scaling_factor=2.5, F_shared=2048, seed=24)
-    hidden, ids, w, weights = _inputs(cfg)
-    out, _ = _run(cfg, hidden, ids, w, weights)
-    # tables (2) + gather + gate+up with the shared gate+up + routed down +
-    # shared down + unpermute
-    assert M.moe_last_launch_count() == 7
-    ref = _oracle(cfg, hidden, ids, w, weights)
-    gu.assert_within_tol(gu.f64(out), ref, cfg.name)
-
-
-def test_shared_expert_launches_on_the_headline_workload():
-    """DeepSeek-V3 prefill: both shared GEMMs share their routed counterpart's
-    launch (tables 2, gather, gate+up, down, unpermute)."""
-    import moe_routed_expert_top_b200 as M
-    cfg = get_config("dsv3_prefill")
-    hidden, ids, w, weights = _inputs(cfg)
-    _run(cfg, hidden, ids, w, weights)
-    assert M.moe_last_launch_count() == 6
-
-
 @pytest.mark.parametrize("name", [n for n in CONFIGS if CONFIGS[n].down_fp8])
 def test_forward_fp8_full_size_sampled(name):
     """The FP8 forward at full size on >= 256 seeded tokens, step by step
