@@ -108,7 +108,8 @@ def work_model(cfg, ids: np.ndarray) -> dict:
     total_bytes = w_gu + w_dn + w_sh + act
     # gate+up kernel alone: its weights, its A rows (x_perm), its h output
     gu_bytes = w_gu + P * H * 2 + P * F * (1 if cfg.down_fp8 else 2) + (P * (F // 128) * 4 if cfg.down_fp8 else 0)
-    dn_bytes = w_dn + P * F * (1 if cfg.down_fp8 else 2) + P * H * 4
+    # the down GEMM writes y in the f16e format (fp16 + an int8 per 128 columns)
+    dn_bytes = w_dn + P * F * (1 if cfg.down_fp8 else 2) + P * H * 2 + P * (H // 128)
     return dict(touched=touched, flops=flops_routed + flops_shared, flops_routed=flops_routed,
                 bytes=total_bytes, gate_up_bytes=gu_bytes, gate_up_flops=4.0 * P * H * F,
                 down_bytes=dn_bytes, down_flops=2.0 * P * H * F)
@@ -229,7 +230,8 @@ def stage_breakdown(M, layer, cfg, hidden, ids, weights, steps, flush):
     else:
         h = torch.empty(P, cfg.F, dtype=torch.bfloat16, device=dev)
         hs = None
-    y = torch.empty(P, cfg.H, dtype=torch.float32, device=dev)
+    y = torch.empty(P, cfg.H, dtype=torch.float16, device=dev)          # f16e, as the forward
+    y_exp = torch.empty(P, cfg.H // 128, dtype=torch.int8, device=dev)
     out = torch.empty(T, cfg.H, dtype=torch.bfloat16, device=dev)
     addend = None
     if cfg.F_shared:
@@ -244,7 +246,7 @@ def stage_breakdown(M, layer, cfg, hidden, ids, weights, steps, flush):
             M.MOE_EPI_SWIGLU_FP8 if cfg.down_fp8 else M.MOE_EPI_SWIGLU, h, hs, None, status),
         "down_gemm": lambda: M.moe_grouped_gemm(
             prob, 0, cfg.H, cfg.F, h, hs, layer.w_down, layer.w_down_scales, tables,
-            M.MOE_EPI_STORE_F32, y, None, None, status),
+            M.MOE_EPI_STORE_F16E, y, y_exp, None, status),
     }
     if cfg.F_shared:
         stages["shared_gate_up_gemm"] = lambda: M.moe_grouped_gemm(
@@ -253,8 +255,8 @@ def stage_breakdown(M, layer, cfg, hidden, ids, weights, steps, flush):
         stages["shared_down_gemm"] = lambda: M.moe_grouped_gemm(
             None, T, cfg.H, cfg.F_shared, sh, None, layer.ws_down, None, None,
             M.MOE_EPI_STORE_F32, addend, None, None, status)
-    stages["unpermute"] = lambda: M.moe_unpermute(prob, y, tables, weights,
-                                                  cfg.routed_scaling_factor, addend, out)
+    stages["unpermute"] = lambda: M.moe_unpermute_f16e(prob, y, y_exp, tables, weights,
+                                                       cfg.routed_scaling_factor, addend, out)
     stream = torch.cuda.current_stream()
     res = {}
     for name, fn in stages.items():

@@ -92,7 +92,10 @@ enum {
   MOE_EPI_STORE = 0,       /* C bf16 [rows, N] = A @ B^T */
   MOE_EPI_SWIGLU = 1,      /* C bf16 [rows, N/2] = SiLU(G[:, :N/2]) * G[:, N/2:] */
   MOE_EPI_SWIGLU_FP8 = 2,  /* C e4m3 [rows, N/2] + C_scales fp32 [rows, N/256] */
-  MOE_EPI_STORE_F32 = 3    /* C fp32 [rows, N] = A @ B^T (the accumulator, unrounded) */
+  MOE_EPI_STORE_F32 = 3,   /* C fp32 [rows, N] = A @ B^T (the accumulator, unrounded) */
+  MOE_EPI_STORE_F16E = 4   /* C fp16 [rows, N] and one int8 exponent per row and 128
+                              columns in C_scales (read as int8_t [rows, N/128]):
+                              A @ B^T = C * 2^e (see moe_unpermute_f16e) */
 };
 
 /* Tiling choice, OR-ed into moe_grouped_gemm's `epilogue` argument. Both
@@ -233,6 +236,11 @@ moe_status moe_route_permute(const moe_problem* prob, const float* logits,
  *   C [rows, N] = sum over K-blocks kb of sa[r,kb]*sb[n/128,kb]*(A_kb @ B_kb^T),
  *   bf16 with MOE_EPI_STORE or fp32 with MOE_EPI_STORE_F32; N % 128 == 0,
  *   K % 128 == 0.
+ * MOE_EPI_STORE_F16E (bf16 or FP8 operands): C fp16 [rows, N] and int8
+ *   exponents in C_scales [rows, N/128], result = C * 2^e per row and
+ *   128-column block (see moe_unpermute_f16e); N % 128 == 0; the weight-row
+ *   and weight-row pair tilings only (MOE_TILE_TOKEN_ROWS, or an automatic
+ *   choice of it: MOE_ERR_UNSUPPORTED).
  * Device flags: MOE_DEV_TIMEOUT into *dev_status (required). */
 moe_status moe_grouped_gemm(const moe_problem* prob, int32_t M_rows, int32_t N, int32_t K,
                             const void* A, const float* A_scales,
@@ -260,6 +268,21 @@ moe_status moe_swiglu_quant(int32_t M, int32_t F, const void* gate_up, const flo
 moe_status moe_unpermute(const moe_problem* prob, const float* y, const int32_t* tables,
                          const float* topk_weights, float scale, const float* addend,
                          void* out, moe_stream_t stream);
+
+/* a7 from the down GEMM's MOE_EPI_STORE_F16E output (no counterpart on the
+ * pages, which hand a bf16 y to the unpermute): y16 fp16 [P, H] and y_exp int8
+ * [P, H/128] with y[r, c] = y16[r, c] * 2^y_exp[r, c/128]. The exponent of a
+ * row's 128-column block puts the block's largest magnitude in [2^14, 2^15),
+ * so every value keeps 11 significant bits (8x bf16's precision) at any fp32
+ * range, in half the bytes of fp32; moe_experts_forward stores y this way when
+ * its down GEMM's tiling supports it. Otherwise as moe_unpermute: each row is
+ * decoded exactly to fp32, then out[t] = RNE_bf16(scale * sum_j w[t,j] *
+ * y[row_of_pair[t*k+j]] + addend[t]) with fp32 sums in slot order. Needs
+ * H % 128 == 0 and 16-byte-aligned y16, out and addend, else
+ * MOE_ERR_INVALID_ARG. */
+moe_status moe_unpermute_f16e(const moe_problem* prob, const void* y16, const int8_t* y_exp,
+                              const int32_t* tables, const float* topk_weights, float scale,
+                              const float* addend, void* out, moe_stream_t stream);
 
 /* a6 with the routing weight folded into the epilogue ([PR1580] Unpermute's
  * scale folding, applied one step earlier, as the down projection's per-row

@@ -22,7 +22,7 @@ __all__ = [
     "moe_dual_blocks", "moe_quant_dual", "moe_swiglu_quant_dual", "moe_swiglu_backward",
     "moe_ep_split_ids", "moe_gather_rows", "moe_down_gemm_weighted", "moe_combine",
     "moe_experts_forward_noalloc", "moe_noalloc_read_status", "moe_selftest_bounded_wait",
-    "EXPORTED_SYMBOLS",
+    "moe_unpermute_f16e", "EXPORTED_SYMBOLS",
     "MOE_OK", "MOE_EPI_STORE", "MOE_EPI_SWIGLU", "MOE_EPI_SWIGLU_FP8", "MOE_EPI_STORE_F32",
     "MOE_SCORE_SOFTMAX", "MOE_SCORE_SIGMOID", "MOE_DEV_BAD_EXPERT_ID", "MOE_DEV_TIMEOUT",
 ]
@@ -36,6 +36,7 @@ MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_DEVICE_FLAG = -4, -5, -6
 MOE_DEV_BAD_EXPERT_ID, MOE_DEV_TIMEOUT, MOE_DEV_BAD_TABLES = 1, 2, 4
 MOE_SCORE_SOFTMAX, MOE_SCORE_SIGMOID = 0, 1
 MOE_EPI_STORE, MOE_EPI_SWIGLU, MOE_EPI_SWIGLU_FP8, MOE_EPI_STORE_F32 = 0, 1, 2, 3
+MOE_EPI_STORE_F16E = 4
 MOE_TILE_AUTO, MOE_TILE_TOKEN_ROWS, MOE_TILE_WEIGHT_ROWS = 0x00, 0x10, 0x20
 MOE_TILE_WEIGHT_ROWS_PAIR = 0x30
 MOE_A_GATHER = 0x100  # moe_grouped_gemm: A = hidden states, rows gathered through the tables
@@ -49,7 +50,7 @@ EXPORTED_SYMBOLS = (
     "moe_shared_workspace_bytes", "moe_shared_expert_forward",
     "moe_dual_blocks", "moe_quant_dual", "moe_swiglu_quant_dual", "moe_swiglu_backward",
     "moe_ep_split_ids", "moe_gather_rows", "moe_down_gemm_weighted", "moe_combine",
-    "moe_noalloc_read_status", "moe_selftest_bounded_wait",
+    "moe_noalloc_read_status", "moe_selftest_bounded_wait", "moe_unpermute_f16e",
 )
 
 
@@ -117,6 +118,7 @@ def lib() -> ctypes.CDLL:
         "moe_swiglu_quant": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, _P, _P,
                                             ctypes.c_int32, _P, _P, _P]),
         "moe_unpermute": (ctypes.c_int, [PP, _P, _P, _P, ctypes.c_float, _P, _P, _P]),
+        "moe_unpermute_f16e": (ctypes.c_int, [PP, _P, _P, _P, _P, ctypes.c_float, _P, _P, _P]),
         "moe_down_gemm_weighted": (ctypes.c_int, [PP, ctypes.c_int32, ctypes.c_int32, _P, _P,
                                                   _P, _P, _P, _P, ctypes.c_float, ctypes.c_int32,
                                                   _P, _P, _P]),
@@ -230,6 +232,12 @@ def moe_unpermute(prob, y, tables, topk_weights, scale, addend, out, stream=None
     _check(lib().moe_unpermute(ctypes.byref(prob), _ptr(y), _ptr(tables), _ptr(topk_weights),
                                float(scale), _ptr(addend), _ptr(out), _stream(stream)),
            "moe_unpermute")
+
+
+def moe_unpermute_f16e(prob, y16, y_exp, tables, topk_weights, scale, addend, out, stream=None):
+    _check(lib().moe_unpermute_f16e(ctypes.byref(prob), _ptr(y16), _ptr(y_exp), _ptr(tables),
+                                    _ptr(topk_weights), float(scale), _ptr(addend), _ptr(out),
+                                    _stream(stream)), "moe_unpermute_f16e")
 
 
 def moe_down_gemm_weighted(prob, N, K, A, A_scales, B, B_scales, tables, topk_weights, scale,

@@ -80,7 +80,8 @@ void fill_layout(const moe_problem* pr, moe_tables_layout* L) {
 }
 
 struct WorkspacePlan {
-  int64_t status = 0, tables = 0, x_perm = 0, h = 0, h_scales = 0, y = 0, hs = 0, ys = 0, total = 0;
+  int64_t status = 0, tables = 0, x_perm = 0, h = 0, h_scales = 0, y = 0, y_exp = 0, hs = 0, ys = 0,
+          total = 0;
 };
 
 WorkspacePlan plan_workspace(const moe_problem* pr) {
@@ -99,7 +100,10 @@ WorkspacePlan plan_workspace(const moe_problem* pr) {
   w.x_perm = take(P * H * 2);
   w.h = take(P * F * (pr->down_fp8 ? 1 : 2));
   w.h_scales = take(pr->down_fp8 ? P * (F / 128) * 4 : 0);
-  w.y = take(P * H * 4);               // fp32: the down GEMM's accumulator, unrounded
+  // the down GEMM's output: fp32 [P, H], or f16e (fp16 [P, H] in the same
+  // region + int8 exponents [P, H/128])
+  w.y = take(P * H * 4);
+  w.y_exp = take(P * ((H + 127) / 128));
   w.hs = take(Fs ? T * Fs * 2 : 0);
   w.ys = take(Fs ? T * H * 4 : 0);
   w.total = o;
@@ -211,8 +215,17 @@ moe_status moe_grouped_gemm(const moe_problem* prob, int32_t M_rows, int32_t N, 
     g.E = 1;
   }
   if (g.rows == 0) return MOE_OK;
+  if (epilogue == MOE_EPI_STORE_F16E) {
+    // fp16 + one int8 exponent per row and 128 columns, into C and C_scales
+    if (C_scales == nullptr) return MOE_ERR_INVALID_ARG;
+    if (N % 128 != 0) return MOE_ERR_UNSUPPORTED;
+    g.out_f16e = 1;
+    g.C_exps = reinterpret_cast<int8_t*>(C_scales);
+  }
   if (fp8) {
-    if (epilogue != MOE_EPI_STORE && epilogue != MOE_EPI_STORE_F32) return MOE_ERR_UNSUPPORTED;
+    if (epilogue != MOE_EPI_STORE && epilogue != MOE_EPI_STORE_F32 &&
+        epilogue != MOE_EPI_STORE_F16E)
+      return MOE_ERR_UNSUPPORTED;
     if (N % 128 != 0 || K % 128 != 0) return MOE_ERR_UNSUPPORTED;
     g.mode = moe::kModeFp8Store;
     g.out_f32 = epilogue == MOE_EPI_STORE_F32;
@@ -221,6 +234,7 @@ moe_status moe_grouped_gemm(const moe_problem* prob, int32_t M_rows, int32_t N, 
     switch (epilogue) {
       case MOE_EPI_STORE:
       case MOE_EPI_STORE_F32:
+      case MOE_EPI_STORE_F16E:
         if (N % 64 != 0) return MOE_ERR_UNSUPPORTED;
         g.mode = moe::kModeStore;
         g.out_f32 = epilogue == MOE_EPI_STORE_F32;
@@ -253,6 +267,7 @@ moe_status moe_grouped_gemm(const moe_problem* prob, int32_t M_rows, int32_t N, 
     return MOE_ERR_UNSUPPORTED;
   if (g.tiling == moe::kTilingWeightsPair && !moe::grouped_gemm_pair_supported(g))
     return MOE_ERR_UNSUPPORTED;
+  if (g.out_f16e && !moe::grouped_gemm_f16e_supported(g)) return MOE_ERR_UNSUPPORTED;
   // gathering is built into the weight-row pair tiling only
   if (g.gather && ((g.tiling != moe::kTilingAuto && g.tiling != moe::kTilingWeightsPair) ||
                    !moe::grouped_gemm_pair_supported(g)))
@@ -291,6 +306,25 @@ moe_status moe_unpermute(const moe_problem* prob, const float* y, const int32_t*
   MOE_CUDA_TRY(moe::launch_unpermute(y, tables + L.row_of_pair, topk_weights, prob->T,
                                      prob->top_k, prob->H, scale, addend, out,
                                      reinterpret_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_unpermute_f16e(const moe_problem* prob, const void* y16, const int8_t* y_exp,
+                              const int32_t* tables, const float* topk_weights, float scale,
+                              const float* addend, void* out, moe_stream_t stream) {
+  moe_status s = check_problem(prob, false);
+  if (s != MOE_OK) return s;
+  if (prob->T == 0) return MOE_OK;
+  if (y16 == nullptr || y_exp == nullptr || tables == nullptr || topk_weights == nullptr ||
+      out == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (prob->H % 128 != 0 || !aligned16(y16) || !aligned16(out) || (addend && !aligned16(addend)))
+    return MOE_ERR_INVALID_ARG;
+  moe_tables_layout L;
+  fill_layout(prob, &L);
+  MOE_CUDA_TRY(moe::launch_unpermute_f16e(y16, y_exp, tables + L.row_of_pair, topk_weights,
+                                          prob->T, prob->top_k, prob->H, scale, addend, out,
+                                          reinterpret_cast<cudaStream_t>(stream)));
   return MOE_OK;
 }
 
@@ -460,9 +494,19 @@ moe_status moe_experts_forward(const moe_problem* prob, const void* hidden,
   g.B = w_down;
   g.A_scales = prob->down_fp8 ? h_scales : nullptr;
   g.B_scales = prob->down_fp8 ? w_down_scales : nullptr;
-  g.C = y;
-  g.out_f32 = 1;
   g.C_scales = nullptr;
+  // y in f16e (half the bytes of fp32, 11 significant bits per value) where the
+  // down GEMM's tiling stores it, else fp32
+  int8_t* y_exp = reinterpret_cast<int8_t*>(base + w.y_exp);
+  g.C = y;
+  g.out_f16e = 1;
+  g.C_exps = y_exp;
+  const bool f16e = moe::grouped_gemm_f16e_supported(g);
+  if (!f16e) {
+    g.out_f16e = 0;
+    g.C_exps = nullptr;
+    g.out_f32 = 1;
+  }
   MOE_CUDA_TRY(moe::launch_grouped_gemm(g, st));
   g_last_launches += 2;
 
@@ -492,8 +536,12 @@ moe_status moe_experts_forward(const moe_problem* prob, const void* hidden,
     g_last_launches += 2;
   }
   // a7
-  MOE_CUDA_TRY(moe::launch_unpermute(y, tables + L.row_of_pair, topk_weights, T, k, H, scale,
-                                     addend, out, st));
+  if (f16e)
+    MOE_CUDA_TRY(moe::launch_unpermute_f16e(y, y_exp, tables + L.row_of_pair, topk_weights, T, k,
+                                            H, scale, addend, out, st));
+  else
+    MOE_CUDA_TRY(moe::launch_unpermute(y, tables + L.row_of_pair, topk_weights, T, k, H, scale,
+                                       addend, out, st));
   g_last_launches += 1;
   return MOE_OK;
 }

@@ -7,6 +7,7 @@
 
 #include <cstdint>
 
+#include "f16e.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -98,6 +99,89 @@ cudaError_t launch_unpermute(const float* y, const int32_t* row_of_pair, const f
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   unpermute_kernel<<<static_cast<unsigned>(blocks), 128, 0, stream>>>(
       reinterpret_cast<const float4*>(y), row_of_pair, weights, k, T * k, H8, scale,
+      reinterpret_cast<const float4*>(addend), static_cast<uint4*>(out), cblocks);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// a7 from the down GEMM's f16e rows (f16e.cuh): y = y16 * 2^e with one int8
+// exponent per row and 128-column block. Each row is decoded to its fp32
+// value (exact) before the same fp32 sums in slot order as above; the row
+// reads are 16 bytes per 8 columns instead of 32.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) unpermute_f16e_kernel(
+    const uint4* __restrict__ y16, const int8_t* __restrict__ y_exp,
+    const int32_t* __restrict__ row_of_pair, const float* __restrict__ w, int k, int P, int H8,
+    float scale, const float4* __restrict__ addend, uint4* __restrict__ out, int cblocks) {
+  const int t = static_cast<int>(blockIdx.x / cblocks);
+  const int c = static_cast<int>(blockIdx.x % cblocks) * blockDim.x + threadIdx.x;  // 8-column group
+  if (c >= H8) return;
+  const int HB = H8 / 16;  // 128-column blocks per row
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+  const int64_t pbase = static_cast<int64_t>(t) * k;
+  for (int j0 = 0; j0 < k; j0 += 8) {
+    int rows[8];
+    float wts[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const bool in = j0 + j < k;
+      const int r = in ? __ldg(row_of_pair + pbase + j0 + j) : -1;
+      rows[j] = (r >= 0 && r < P) ? r : -1;
+      wts[j] = in ? __ldg(w + pbase + j0 + j) : 0.0f;
+    }
+    uint4 va[8];
+    int ex[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (rows[j] >= 0) {
+        va[j] = __ldg(y16 + static_cast<int64_t>(rows[j]) * H8 + c);
+        ex[j] = __ldg(y_exp + static_cast<int64_t>(rows[j]) * HB + (c >> 4));
+      } else {
+        va[j] = make_uint4(0u, 0u, 0u, 0u);
+        ex[j] = 0;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (j0 + j >= k) break;
+      if (rows[j] < 0) continue;
+      const float s2 = f16e_pow2(ex[j]);
+      const uint32_t wd[4] = {va[j].x, va[j].y, va[j].z, va[j].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wd[q]));
+        acc[2 * q] = fmaf(wts[j], f.x * s2, acc[2 * q]);
+        acc[2 * q + 1] = fmaf(wts[j], f.y * s2, acc[2 * q + 1]);
+      }
+    }
+  }
+  float v[8];
+  if (addend != nullptr) {
+    const float4* ad = addend + (static_cast<int64_t>(t) * H8 + c) * 2;
+    const float4 a = __ldg(ad), b = __ldg(ad + 1);
+    const float add[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = fmaf(scale, acc[i], add[i]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = scale * acc[i];
+  }
+  out[static_cast<int64_t>(t) * H8 + c] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                                     pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+}
+
+cudaError_t launch_unpermute_f16e(const void* y16, const int8_t* y_exp, const int32_t* row_of_pair,
+                                  const float* weights, int T, int k, int H, float scale,
+                                  const float* addend, void* out, cudaStream_t stream) {
+  if (T <= 0) return cudaSuccess;
+  const int H8 = H / 8;
+  const int cblocks = (H8 + 127) / 128;
+  const long long blocks = static_cast<long long>(T) * cblocks;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  unpermute_f16e_kernel<<<static_cast<unsigned>(blocks), 128, 0, stream>>>(
+      static_cast<const uint4*>(y16), y_exp, row_of_pair, weights, k, T * k, H8, scale,
       reinterpret_cast<const float4*>(addend), static_cast<uint4*>(out), cblocks);
   return cudaGetLastError();
 }

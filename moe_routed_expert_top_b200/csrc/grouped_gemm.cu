@@ -643,8 +643,9 @@ cudaError_t launch_grouped_gemm(const GemmLaunch& L, cudaStream_t stream) {
       (L.tiling == kTilingWeights || (L.tiling == kTilingAuto && grouped_gemm_t_preferred(L))))
     return launch_grouped_gemm_t(L, stream);
   if (L.tiling == kTilingWeights) return cudaErrorNotSupported;
-  // the weighted (pair-order) store is built into the weight-row tilings only
-  if (L.weighted) return cudaErrorNotSupported;
+  // the weighted (pair-order) store and the f16e format are built into the
+  // weight-row tilings only
+  if (L.weighted || L.out_f16e) return cudaErrorNotSupported;
   switch (L.mode) {
     case kModeStore:
       if (L.N % 256 == 0) return run_gemm<kModeStore, 256>(L, stream);
@@ -665,6 +666,21 @@ cudaError_t launch_grouped_gemm(const GemmLaunch& L, cudaStream_t stream) {
     default:
       return cudaErrorInvalidValue;
   }
+}
+
+}  // namespace moe
+
+namespace moe {
+
+bool grouped_gemm_f16e_supported(const GemmLaunch& L) {
+  if (!L.out_f16e) return false;
+  // the dispatch of launch_grouped_gemm, for a launch that stores f16e
+  const bool b_view = L.ldb != 0 || L.up_off != 0 || L.b_rows != 0;
+  if (L.gather || b_view || L.tiling == kTilingWeightsPair ||
+      (L.tiling == kTilingAuto && grouped_gemm_pair_preferred(L)))
+    return grouped_gemm_pair_supported(L);
+  return grouped_gemm_t_supported(L) &&
+         (L.tiling == kTilingWeights || (L.tiling == kTilingAuto && grouped_gemm_t_preferred(L)));
 }
 
 }  // namespace moe

@@ -32,6 +32,7 @@
 
 #include <mutex>
 
+#include "f16e.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -54,6 +55,8 @@ struct TParams {
   void* C;
   int ldc;      // output row length in elements
   int out_f32;  // store modes: fp32 C
+  int out_f16e;     // store modes: C fp16 + C_exps int8 [rows, ldc / 128] (f16e.cuh)
+  int8_t* C_exps;
   const float* A_scales;  // FP8: activation scales [rows, KBS]
   const float* B_scales;  // FP8: weight block scales [E, N/128, KBS]
   int KBS;                // FP8: K / 128
@@ -157,11 +160,32 @@ __device__ __forceinline__ void stage_row_info(const TParams& p, int et, int row
 }
 
 // Write `rows` staged token rows (sOut[i][0..128), fp32) to C rows row0.. at
-// column col0, fp32 or bf16, 16-byte stores; 128 epilogue threads (et). A
+// column col0, fp32, bf16 or f16e, 16-byte stores; 128 epilogue threads (et). A
 // weighted store writes row i to sDst[i], scaled by sFac[i].
 __device__ __forceinline__ void store_rows(const TParams& p, const float* sOut, int et, int rows,
                                            int row0, int col0, const int* sDst,
                                            const float* sFac) {
+  if (p.out_f16e) {
+    // a row's 128 columns (one f16e block) over 16 lanes of a half warp; every
+    // lane encodes, whether or not its row is stored
+#pragma unroll
+    for (int pass = 0; pass < 4; ++pass) {
+      const int i = pass * 8 + (et >> 4);
+      const int c8 = et & 15;
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = sOut[i * 128 + c8 * 8 + u];
+      uint4 pk;
+      const int e = f16e_encode8(v, pk);
+      if (i < rows) {
+        const int64_t row = row0 + i;
+        __half* dst = static_cast<__half*>(p.C) + row * p.ldc + col0;
+        reinterpret_cast<uint4*>(dst)[c8] = pk;
+        if (c8 == 0) p.C_exps[row * (p.ldc / 128) + col0 / 128] = static_cast<int8_t>(e);
+      }
+    }
+    return;
+  }
   if (p.out_f32) {
 #pragma unroll
     for (int pass = 0; pass < 8; ++pass) {
@@ -719,6 +743,8 @@ cudaError_t run_t(const GemmLaunch& L, cudaStream_t stream) {
   p.C = L.C;
   p.ldc = kMode == kTSwiglu ? L.N / 2 : L.N;
   p.out_f32 = L.out_f32;
+  p.out_f16e = L.out_f16e;
+  p.C_exps = L.C_exps;
   p.A_scales = L.A_scales;
   p.B_scales = L.B_scales;
   p.KBS = L.K / 128;
@@ -742,6 +768,9 @@ cudaError_t run_t(const GemmLaunch& L, cudaStream_t stream) {
 
 bool grouped_gemm_t_supported(const GemmLaunch& L) {
   if (L.E > 1024) return false;
+  if (L.out_f16e && ((L.mode != kModeStore && L.mode != kModeFp8Store) || L.weighted ||
+                     L.out_f32 || L.C_exps == nullptr))
+    return false;
   if (L.weighted && (L.pair_of_row == nullptr || L.row_weights == nullptr ||
                      L.group_sizes == nullptr ||
                      (L.mode != kModeStore && L.mode != kModeFp8Store)))

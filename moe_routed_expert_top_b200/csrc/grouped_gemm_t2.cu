@@ -32,6 +32,7 @@
 
 #include <mutex>
 
+#include "f16e.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -54,6 +55,8 @@ struct PParams {
   void* C;
   int ldc;
   int out_f32;
+  int out_f16e;     // C fp16 + C_exps int8 [rows, ldc / 128] (f16e.cuh)
+  int8_t* C_exps;
   int32_t* status;
   // gather mode: token row r is hidden[pair_of_row[r] / top_k] (K columns)
   const __nv_bfloat16* hidden;
@@ -463,6 +466,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                 reinterpret_cast<float4*>(dst)[c4] = val;
               }
             }
+          } else if (p.out_f16e) {
+            // f16e: a row's 128 columns are this CTA's output block, held by 16
+            // lanes of a half warp (8 columns each); every lane encodes
+#pragma unroll
+            for (int pass = 0; pass < 4; ++pass) {
+              const int i = pass * 8 + (et >> 4);
+              const int c8 = et & 15;
+              float v[8];
+#pragma unroll
+              for (int u = 0; u < 8; ++u) v[u] = sOut[i * 128 + c8 * 8 + u];
+              uint4 pk;
+              const int e = f16e_encode8(v, pk);
+              if (i < rows) {
+                const int64_t row = ti.m0 + j0 + i;
+                __half* dst = static_cast<__half*>(p.C) + row * p.ldc + col0;
+                reinterpret_cast<uint4*>(dst)[c8] = pk;
+                if (c8 == 0) p.C_exps[row * (p.ldc / 128) + col0 / 128] = static_cast<int8_t>(e);
+              }
+            }
           } else {
 #pragma unroll
             for (int pass = 0; pass < 4; ++pass) {
@@ -610,6 +632,8 @@ cudaError_t run_pair(const GemmLaunch& L, cudaStream_t stream) {
   p.C = L.C;
   p.ldc = kMode == kPSwiglu ? L.N / 2 : L.N;
   p.out_f32 = L.out_f32;
+  p.out_f16e = L.out_f16e;
+  p.C_exps = L.C_exps;
   p.status = L.status;
   p.hidden = static_cast<const __nv_bfloat16*>(L.A);
   p.pair_of_row = L.pair_of_row;
@@ -648,6 +672,8 @@ bool grouped_gemm_pair_supported(const GemmLaunch& L) {
     return false;
   // a strided view of B: rows at least K long, 16-byte row pitch
   if (L.ldb != 0 && (L.ldb < L.K || L.ldb % 8 != 0)) return false;
+  if (L.out_f16e && (L.mode != kModeStore || L.weighted || L.out_f32 || L.C_exps == nullptr))
+    return false;
   if (L.mode == kModeStore) return L.N % 256 == 0 && L.K % 64 == 0 && L.up_off == 0;
   if (L.mode == kModeSwiglu) return (L.N / 2) % 128 == 0 && L.K % 64 == 0;
   return false;

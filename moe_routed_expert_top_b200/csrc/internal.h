@@ -29,6 +29,11 @@ struct GemmLaunch {
   int M_blk = 0;  // length of idx_for_bx (grouped mode)
   void* C = nullptr;
   int out_f32 = 0;  // store modes: fp32 C instead of bf16
+  // store modes: C fp16 with one int8 power-of-two exponent per row and
+  // 128-column block in C_exps [rows, N / 128] (f16e.cuh); weight-row and
+  // pair tilings, not with the weighted store
+  int out_f16e = 0;
+  int8_t* C_exps = nullptr;
   float* C_scales = nullptr;
   float* debug_h = nullptr;
   int32_t* status = nullptr;
@@ -68,6 +73,8 @@ bool grouped_gemm_t_preferred(const GemmLaunch& L);
 cudaError_t launch_grouped_gemm_pair(const GemmLaunch& L, cudaStream_t stream);
 bool grouped_gemm_pair_supported(const GemmLaunch& L);
 bool grouped_gemm_pair_preferred(const GemmLaunch& L);
+// Whether the automatic (or requested) tiling of L stores the f16e format.
+bool grouped_gemm_f16e_supported(const GemmLaunch& L);
 
 cudaError_t launch_route_topk(const float* logits, int T, int E, int k, int score_fn,
                               int renormalize, int32_t* ids, float* weights, cudaStream_t stream);
@@ -86,6 +93,11 @@ cudaError_t launch_gather_rows(const void* hidden, const int32_t* pair_of_row, i
 cudaError_t launch_unpermute(const float* y, const int32_t* row_of_pair, const float* weights,
                              int T, int k, int H, float scale, const float* addend, void* out,
                              cudaStream_t stream);
+// The same from the down GEMM's f16e output: y16 fp16 [T*k, H], y_exp int8
+// [T*k, H/128], y = y16 * 2^y_exp.
+cudaError_t launch_unpermute_f16e(const void* y16, const int8_t* y_exp, const int32_t* row_of_pair,
+                                  const float* weights, int T, int k, int H, float scale,
+                                  const float* addend, void* out, cudaStream_t stream);
 cudaError_t launch_combine(const void* y_w, bool y_f32, const int32_t* row_of_pair, int T, int k,
                            int H, const float* addend, void* out, cudaStream_t stream);
 

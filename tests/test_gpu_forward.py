@@ -248,14 +248,16 @@ def test_forward_fp8_full_size_sampled(name):
     q_ref, s_ref = O.quant_1x128(h_gpu)
     assert np.array_equal(q_gpu, q_ref)
     assert np.array_equal(s_gpu.view(np.uint32), s_ref.view(np.uint32))
-    # (2) the down GEMM + unpermute fed the oracle's codes and scales
-    y = torch.empty(P, H, dtype=torch.float32, device="cuda")
+    # (2) the down GEMM + unpermute fed the oracle's codes and scales, with the
+    # forward's f16e intermediate
+    y16 = torch.empty(P, H, dtype=torch.float16, device="cuda")
+    yex = torch.empty(P, H // 128, dtype=torch.int8, device="cuda")
     M.moe_grouped_gemm(prob, 0, H, F, torch.from_numpy(qa_all).cuda(),
                        torch.from_numpy(sa_all).cuda(), layer.w_down, layer.w_down_scales, tables,
-                       M.MOE_EPI_STORE_F32, y, None, None, status)
+                       M.MOE_EPI_STORE_F16E, y16, yex, None, status)
     out2 = torch.empty(cfg.T, H, dtype=torch.bfloat16, device="cuda")
-    M.moe_unpermute(prob, y, tables, torch.from_numpy(w).cuda(), cfg.routed_scaling_factor,
-                    None, out2)
+    M.moe_unpermute_f16e(prob, y16, yex, tables, torch.from_numpy(w).cuda(),
+                         cfg.routed_scaling_factor, None, out2)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     gu.assert_within_tol(gu.f64(out2)[tokens], ref, f"{name}: down + unpermute on oracle codes")

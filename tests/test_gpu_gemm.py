@@ -416,3 +416,94 @@ def test_swiglu_fp8_epilogue_full_size_bits():
     assert np.array_equal(q.cpu().numpy(), q_ref)
     assert np.array_equal(sc.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
     assert (s_ref > 0).all()
+
+
+def _f16e_decode(c16: torch.Tensor, exps: torch.Tensor) -> np.ndarray:
+    """y = C16 * 2^e per row and 128-column block (exact in float64)."""
+    c = c16.float().cpu().numpy().astype(np.float64)
+    e = exps.cpu().numpy().astype(np.int64)
+    return c * np.repeat(np.ldexp(1.0, e), 128, axis=1)
+
+
+def _check_f16e(dec, ref, what):
+    """Every value within the fp32 store's tolerance of the oracle's (the
+    tensor core's fp32 sums: 1e-4 + 1e-4*|ref|) plus fp16's rounding (11
+    significant bits: 2^-11 relative, and the subnormal step of its block)."""
+    rows, n = ref.shape
+    bmax = np.abs(ref).reshape(rows, n // 128, 128).max(2)
+    step = np.repeat(bmax, 128, axis=1) * 2.0 ** -38
+    err = np.abs(dec - ref)
+    bound = 1e-4 + np.abs(ref) * (1e-4 + 2.0 ** -11) + step
+    assert np.all(err <= bound), (what, float((err / bound).max()))
+
+
+@pytest.mark.parametrize("tiling", TILINGS)
+@pytest.mark.parametrize("T,E,k,H,F,sizes", [(200, 8, 2, 256, 384, None),
+                                            (260, 8, 3, 512, 256, [0, 1, 127, 128, 129, 0, 255, 140]),
+                                            (546, 8, 4, 256, 256, [257, 288, 289, 517, 544, 256, 0, 33])])
+def test_grouped_gemm_store_f16e(T, E, k, H, F, sizes, tiling):
+    """MOE_EPI_STORE_F16E (the forward's down-GEMM output): fp16 values and one
+    int8 exponent per row and 128 columns, decoded against the oracle's
+    float64 product; the token-row tiling refuses it."""
+    gu = _gu()
+    import moe_routed_expert_top_b200 as M
+    cfg, ids, hidden, L, tables, status, x_perm, ref, wgu, wd = _setup(T, E, k, H, F, 6, sizes)
+    prob = gu.problem(cfg)
+    P, N = L["P"], 2 * F
+    c16 = torch.full((P, N), float("nan"), dtype=torch.float16, device="cuda")
+    ex = torch.zeros(P, N // 128, dtype=torch.int8, device="cuda")
+    call = lambda: M.moe_grouped_gemm(prob, 0, N, H, x_perm, None, wgu, None, tables,
+                                      M.MOE_EPI_STORE_F16E | tiling, c16, ex, None, status)
+    if tiling == 0x10 or _pair_unsupported(tiling, N):
+        _expect_unsupported(call)
+        return
+    call()
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    refC = _oracle_rows_gemm(hidden, wgu, ref, E, k)
+    dec = _f16e_decode(c16, ex)
+    _check_f16e(dec, refC, "f16e store")
+    # and, value for value, the same tiling's fp32 store rounded once to fp16
+    # under the block exponent (the encoding is exact apart from that rounding)
+    c32 = torch.empty(P, N, dtype=torch.float32, device="cuda")
+    M.moe_grouped_gemm(prob, 0, N, H, x_perm, None, wgu, None, tables,
+                       M.MOE_EPI_STORE_F32 | tiling, c32, None, None, status)
+    torch.cuda.synchronize()
+    y32 = c32.cpu().numpy().astype(np.float64)
+    scale = np.repeat(np.ldexp(1.0, ex.cpu().numpy().astype(np.int64)), 128, axis=1)
+    assert np.array_equal((y32 / scale).astype(np.float16).astype(np.float64) * scale, dec)
+    # the exponent rule: each block's largest magnitude in [2^14, 2^15] * 2^e
+    e = ex.cpu().numpy().astype(np.int64)
+    cmax = np.abs(c16.float().cpu().numpy()).reshape(P, N // 128, 128).max(2)
+    nz = cmax > 0
+    assert np.all((cmax[nz] >= 2.0 ** 14) & (cmax[nz] <= 2.0 ** 15))
+    assert np.all(e[~nz] == 0)
+
+
+def test_grouped_gemm_fp8_store_f16e():
+    """The FP8 block-scaled down GEMM (weight-row tiling) stores f16e too."""
+    gu = _gu()
+    import moe_routed_expert_top_b200 as M
+    T, E, k, H, F = 200, 8, 2, 256, 384
+    cfg, ids, hidden, L, tables, status, x_perm, ref, wgu, wd = _setup(T, E, k, H, F, 4)
+    prob = gu.problem(cfg)
+    P = L["P"]
+    rng = np.random.default_rng(9)
+    h = (rng.standard_normal((P, F)) * rng.uniform(0.1, 3, (P, 1))).astype(np.float32)
+    qa, sa = O.quant_1x128(h)
+    wq, ws = zip(*[O.quant_weight_128x128(gu.f64(wd[e]).astype(np.float32)) for e in range(E)])
+    wq, ws = np.stack(wq), np.stack(ws)
+    refy = np.zeros((P, H))
+    for e in range(E):
+        a, b = ref["group_offsets"][e], ref["group_offsets"][e + 1]
+        if b > a:
+            refy[a:b] = O.fp8_block_scaled_matmul(qa[a:b], sa[a:b], wq[e], ws[e])
+    c16 = torch.full((P, H), float("nan"), dtype=torch.float16, device="cuda")
+    ex = torch.zeros(P, H // 128, dtype=torch.int8, device="cuda")
+    M.moe_grouped_gemm(prob, 0, H, F, torch.from_numpy(qa).cuda(), torch.from_numpy(sa).cuda(),
+                       torch.from_numpy(wq).cuda(), torch.from_numpy(ws).cuda(), tables,
+                       M.MOE_EPI_STORE_F16E | 0x20, c16, ex, None, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    # the fp32 accumulation of the scaled K-blocks (as the fp32 store) before the fp16 rounding
+    gu.assert_within_tol(_f16e_decode(c16, ex), refy, "fp8 f16e", rtol=1e-3, atol=1e-4)
