@@ -109,7 +109,9 @@ def work_model(cfg, ids: np.ndarray) -> dict:
     # gate+up kernel alone: its weights, its A rows (x_perm), its h output
     gu_bytes = w_gu + P * H * 2 + P * F * (1 if cfg.down_fp8 else 2) + (P * (F // 128) * 4 if cfg.down_fp8 else 0)
     # the down GEMM writes y in the f16e format (fp16 + an int8 per 128 columns)
-    dn_bytes = w_dn + P * F * (1 if cfg.down_fp8 else 2) + P * H * 2 + P * (H // 128)
+    # when F >= 1024, as the forward does, else fp32
+    y_bytes = P * H * 2 + P * (H // 128) if F >= 1024 else P * H * 4
+    dn_bytes = w_dn + P * F * (1 if cfg.down_fp8 else 2) + y_bytes
     return dict(touched=touched, flops=flops_routed + flops_shared, flops_routed=flops_routed,
                 bytes=total_bytes, gate_up_bytes=gu_bytes, gate_up_flops=4.0 * P * H * F,
                 down_bytes=dn_bytes, down_flops=2.0 * P * H * F)
@@ -230,8 +232,10 @@ def stage_breakdown(M, layer, cfg, hidden, ids, weights, steps, flush):
     else:
         h = torch.empty(P, cfg.F, dtype=torch.bfloat16, device=dev)
         hs = None
-    y = torch.empty(P, cfg.H, dtype=torch.float16, device=dev)          # f16e, as the forward
-    y_exp = torch.empty(P, cfg.H // 128, dtype=torch.int8, device=dev)
+    # y as the forward keeps it: f16e when F >= 1024, else fp32
+    f16e = cfg.F >= 1024
+    y = torch.empty(P, cfg.H, dtype=torch.float16 if f16e else torch.float32, device=dev)
+    y_exp = torch.empty(P, cfg.H // 128, dtype=torch.int8, device=dev) if f16e else None
     out = torch.empty(T, cfg.H, dtype=torch.bfloat16, device=dev)
     addend = None
     if cfg.F_shared:
@@ -246,7 +250,7 @@ def stage_breakdown(M, layer, cfg, hidden, ids, weights, steps, flush):
             M.MOE_EPI_SWIGLU_FP8 if cfg.down_fp8 else M.MOE_EPI_SWIGLU, h, hs, None, status),
         "down_gemm": lambda: M.moe_grouped_gemm(
             prob, 0, cfg.H, cfg.F, h, hs, layer.w_down, layer.w_down_scales, tables,
-            M.MOE_EPI_STORE_F16E, y, y_exp, None, status),
+            M.MOE_EPI_STORE_F16E if f16e else M.MOE_EPI_STORE_F32, y, y_exp, None, status),
     }
     if cfg.F_shared:
         stages["shared_gate_up_gemm"] = lambda: M.moe_grouped_gemm(
@@ -255,8 +259,12 @@ def stage_breakdown(M, layer, cfg, hidden, ids, weights, steps, flush):
         stages["shared_down_gemm"] = lambda: M.moe_grouped_gemm(
             None, T, cfg.H, cfg.F_shared, sh, None, layer.ws_down, None, None,
             M.MOE_EPI_STORE_F32, addend, None, None, status)
-    stages["unpermute"] = lambda: M.moe_unpermute_f16e(prob, y, y_exp, tables, weights,
-                                                       cfg.routed_scaling_factor, addend, out)
+    if f16e:
+        stages["unpermute"] = lambda: M.moe_unpermute_f16e(prob, y, y_exp, tables, weights,
+                                                           cfg.routed_scaling_factor, addend, out)
+    else:
+        stages["unpermute"] = lambda: M.moe_unpermute(prob, y, tables, weights,
+                                                      cfg.routed_scaling_factor, addend, out)
     stream = torch.cuda.current_stream()
     res = {}
     for name, fn in stages.items():
