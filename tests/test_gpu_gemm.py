@@ -72,6 +72,9 @@ GEMM_CASES = [
     # evenly over their tiles): 256-token tiles, then 64-token ones
     (546, 8, 4, 256, 256, [257, 288, 289, 517, 544, 256, 0, 33]),
     (256, 8, 2, 256, 256, [65, 96, 97, 160, 64, 0, 1, 29]),
+    # experts averaging <= 160 rows take 192-token pair tiles (96-row token
+    # boxes): one tile up to 192 rows, two above
+    (300, 8, 4, 256, 256, [192, 193, 0, 150, 129, 300, 96, 140]),
 ]
 
 
