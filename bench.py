@@ -108,9 +108,9 @@ def work_model(cfg, ids: np.ndarray) -> dict:
     total_bytes = w_gu + w_dn + w_sh + act
     # gate+up kernel alone: its weights, its A rows (x_perm), its h output
     gu_bytes = w_gu + P * H * 2 + P * F * (1 if cfg.down_fp8 else 2) + (P * (F // 128) * 4 if cfg.down_fp8 else 0)
-    # the down GEMM writes y in the f16e format (fp16 + an int8 per 128 columns)
-    # when F >= 1024, as the forward does, else fp32
-    y_bytes = P * H * 2 + P * (H // 128) if F >= 1024 else P * H * 4
+    # the down GEMM writes y in the f16e format (fp16 + an int8 per 128 columns),
+    # as the forward does on every workload here (its tilings all store f16e)
+    y_bytes = P * H * 2 + P * (H // 128)
     dn_bytes = w_dn + P * F * (1 if cfg.down_fp8 else 2) + y_bytes
     return dict(touched=touched, flops=flops_routed + flops_shared, flops_routed=flops_routed,
                 bytes=total_bytes, gate_up_bytes=gu_bytes, gate_up_flops=4.0 * P * H * F,
@@ -232,8 +232,8 @@ def stage_breakdown(M, layer, cfg, hidden, ids, weights, steps, flush):
     else:
         h = torch.empty(P, cfg.F, dtype=torch.bfloat16, device=dev)
         hs = None
-    # y as the forward keeps it: f16e when F >= 1024, else fp32
-    f16e = cfg.F >= 1024
+    # y as the forward keeps it: f16e (every workload's down tiling stores it)
+    f16e = True
     y = torch.empty(P, cfg.H, dtype=torch.float16 if f16e else torch.float32, device=dev)
     y_exp = torch.empty(P, cfg.H // 128, dtype=torch.int8, device=dev) if f16e else None
     out = torch.empty(T, cfg.H, dtype=torch.bfloat16, device=dev)

@@ -495,18 +495,16 @@ moe_status moe_experts_forward(const moe_problem* prob, const void* hidden,
   g.A_scales = prob->down_fp8 ? h_scales : nullptr;
   g.B_scales = prob->down_fp8 ? w_down_scales : nullptr;
   g.C_scales = nullptr;
-  // y in f16e (half the bytes of fp32, 11 significant bits per value) where the
-  // down GEMM's tiling stores it and its K (= F) is at least 1024, else fp32.
-  // Interleaved A/B of the whole forward on B200: dsv3_prefill (F 2048) 2.1%
-  // faster, Kimi-K2 0.6%, dsv3_decode_fp8 and qwen3_decode even; qwen3_prefill
-  // (F 768) 5.8% slower: on a short K the down GEMM's epilogue, which also
-  // encodes, is on the critical path, and the encoding costs more than the
-  // halved bytes save.
+  // y in f16e (half the bytes of fp32, 11 significant bits per value) wherever
+  // the down GEMM's tiling stores it, else fp32. Down GEMM + unpermute on B200,
+  // f16e against fp32 (us): qwen3_prefill 136 + 42 vs 136 + 60, qwen3_decode
+  // 77 + 12 vs 83 + 15, dsv3_decode_fp8 552 + 23 vs 548 + 33, dsv3_prefill
+  // 1381 + 124 vs 1406 + 173.
   int8_t* y_exp = reinterpret_cast<int8_t*>(base + w.y_exp);
   g.C = y;
   g.out_f16e = 1;
   g.C_exps = y_exp;
-  const bool f16e = F >= 1024 && moe::grouped_gemm_f16e_supported(g);
+  const bool f16e = moe::grouped_gemm_f16e_supported(g);
   if (!f16e) {
     g.out_f16e = 0;
     g.C_exps = nullptr;

@@ -29,27 +29,38 @@ __device__ __forceinline__ float f16e_pow2(int x) {
   return __uint_as_float(static_cast<uint32_t>(x + 127) << 23);
 }
 
-// Encodes 8 consecutive values of one row. The row's 128-column block is
-// spread over 16 consecutive lanes of a half warp (8 columns each); every lane
-// of the warp must call this (the two half warps may encode different rows).
-// Returns the block's exponent (the same in all 16 lanes) and the 8 fp16 codes.
-__device__ __forceinline__ int f16e_encode8(const float (&v)[8], uint4& out) {
-  float amax = 0.0f;
+// Encodes four rows' blocks at once (the four row passes of a 32-row slab).
+// Each row's 128-column block is spread over 16 consecutive lanes of a half
+// warp, 8 columns each (v[q]: this lane's 8 values of pass q); every lane of
+// the warp must call this. Returns each block's exponent (the same in its 16
+// lanes) and this lane's 8 fp16 codes per pass. The four half-warp reductions
+// are interleaved so that their shuffle latencies overlap.
+__device__ __forceinline__ void f16e_encode8x4(const float (&v)[4][8], uint4 (&out)[4],
+                                               int (&e)[4]) {
+  float amax[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  for (int q = 0; q < 4; ++q) {
+    amax[q] = 0.0f;
 #pragma unroll
-  for (int off = 8; off > 0; off >>= 1)
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-  const int e = f16e_exponent(amax);
-  const float s = f16e_pow2(-e);
-  uint32_t w[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const __half2 h = __floats2half2_rn(v[2 * i] * s, v[2 * i + 1] * s);
-    w[i] = *reinterpret_cast<const uint32_t*>(&h);
+    for (int i = 0; i < 8; ++i) amax[q] = fmaxf(amax[q], fabsf(v[q][i]));
   }
-  out = make_uint4(w[0], w[1], w[2], w[3]);
-  return e;
+#pragma unroll
+  for (int off = 8; off > 0; off >>= 1) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) amax[q] = fmaxf(amax[q], __shfl_xor_sync(0xffffffffu, amax[q], off));
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    e[q] = f16e_exponent(amax[q]);
+    const float s = f16e_pow2(-e[q]);
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __half2 h = __floats2half2_rn(v[q][2 * i] * s, v[q][2 * i + 1] * s);
+      w[i] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    out[q] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
 }
 
 }  // namespace moe

@@ -168,20 +168,26 @@ __device__ __forceinline__ void store_rows(const TParams& p, const float* sOut, 
   if (p.out_f16e) {
     // a row's 128 columns (one f16e block) over 16 lanes of a half warp; every
     // lane encodes, whether or not its row is stored
+    const int c8 = et & 15;
+    float v[4][8];
+#pragma unroll
+    for (int pass = 0; pass < 4; ++pass) {
+      const float4* src = reinterpret_cast<const float4*>(sOut + (pass * 8 + (et >> 4)) * 128 + c8 * 8);
+      const float4 a = src[0], b = src[1];
+      v[pass][0] = a.x; v[pass][1] = a.y; v[pass][2] = a.z; v[pass][3] = a.w;
+      v[pass][4] = b.x; v[pass][5] = b.y; v[pass][6] = b.z; v[pass][7] = b.w;
+    }
+    uint4 pk[4];
+    int e[4];
+    f16e_encode8x4(v, pk, e);
 #pragma unroll
     for (int pass = 0; pass < 4; ++pass) {
       const int i = pass * 8 + (et >> 4);
-      const int c8 = et & 15;
-      float v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = sOut[i * 128 + c8 * 8 + u];
-      uint4 pk;
-      const int e = f16e_encode8(v, pk);
       if (i < rows) {
         const int64_t row = row0 + i;
         __half* dst = static_cast<__half*>(p.C) + row * p.ldc + col0;
-        reinterpret_cast<uint4*>(dst)[c8] = pk;
-        if (c8 == 0) p.C_exps[row * (p.ldc / 128) + col0 / 128] = static_cast<int8_t>(e);
+        reinterpret_cast<uint4*>(dst)[c8] = pk[pass];
+        if (c8 == 0) p.C_exps[row * (p.ldc / 128) + col0 / 128] = static_cast<int8_t>(e[pass]);
       }
     }
     return;

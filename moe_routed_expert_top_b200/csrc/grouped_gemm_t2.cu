@@ -469,20 +469,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           } else if (p.out_f16e) {
             // f16e: a row's 128 columns are this CTA's output block, held by 16
             // lanes of a half warp (8 columns each); every lane encodes
+            const int c8 = et & 15;
+            float fv[4][8];
+#pragma unroll
+            for (int pass = 0; pass < 4; ++pass) {
+              const float4* src =
+                  reinterpret_cast<const float4*>(sOut + (pass * 8 + (et >> 4)) * 128 + c8 * 8);
+              const float4 a = src[0], b = src[1];
+              fv[pass][0] = a.x; fv[pass][1] = a.y; fv[pass][2] = a.z; fv[pass][3] = a.w;
+              fv[pass][4] = b.x; fv[pass][5] = b.y; fv[pass][6] = b.z; fv[pass][7] = b.w;
+            }
+            uint4 pk[4];
+            int e[4];
+            f16e_encode8x4(fv, pk, e);
 #pragma unroll
             for (int pass = 0; pass < 4; ++pass) {
               const int i = pass * 8 + (et >> 4);
-              const int c8 = et & 15;
-              float v[8];
-#pragma unroll
-              for (int u = 0; u < 8; ++u) v[u] = sOut[i * 128 + c8 * 8 + u];
-              uint4 pk;
-              const int e = f16e_encode8(v, pk);
               if (i < rows) {
                 const int64_t row = ti.m0 + j0 + i;
                 __half* dst = static_cast<__half*>(p.C) + row * p.ldc + col0;
-                reinterpret_cast<uint4*>(dst)[c8] = pk;
-                if (c8 == 0) p.C_exps[row * (p.ldc / 128) + col0 / 128] = static_cast<int8_t>(e);
+                reinterpret_cast<uint4*>(dst)[c8] = pk[pass];
+                if (c8 == 0)
+                  p.C_exps[row * (p.ldc / 128) + col0 / 128] = static_cast<int8_t>(e[pass]);
               }
             }
           } else {
