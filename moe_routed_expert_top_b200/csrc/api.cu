@@ -6,6 +6,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "internal.h"
 #include "moe.h"
@@ -54,6 +55,45 @@ moe_status check_problem(const moe_problem* pr, bool need_gemm) {
 }
 
 int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
+
+// A second stream per device on which the forward runs the shared expert beside
+// the routed GEMMs (created on first use; null if that fails, and the forward
+// then runs everything on the caller's stream).
+cudaStream_t side_stream() {
+  static cudaStream_t streams[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (streams[dev] == nullptr) {
+    cudaStream_t t = nullptr;
+    if (cudaStreamCreateWithFlags(&t, cudaStreamNonBlocking) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    streams[dev] = t;
+  }
+  return streams[dev];
+}
+
+// SMs given to the shared expert while the routed GEMMs run on the others, so
+// that both finish at about the same time: the shared MLP is compute-bound
+// (its FLOPs at about 0.9 PFLOP/s, the dense rate its tiles reach on B200),
+// the routed GEMMs stream the touched experts' weights at about 5.8 TB/s.
+// Even (the shared GEMMs run on CTA pairs), at least 2, at most a quarter.
+int shared_sms(const moe_problem* pr, int sms) {
+  const double shared_s = 6.0 * pr->T * static_cast<double>(pr->H) * pr->F_shared / 0.9e15;
+  const double touched = pr->E < static_cast<int64_t>(pr->T) * pr->top_k
+                             ? pr->E
+                             : static_cast<double>(pr->T) * pr->top_k;
+  const double routed_s = touched * 3.0 * pr->H * static_cast<double>(pr->F) *
+                          (pr->down_fp8 ? 1.67 : 2.0) / 5.8e12;
+  int k = static_cast<int>(sms * shared_s / (routed_s > 0 ? routed_s : 1e-9) + 0.5);
+  k &= ~1;
+  if (k < 2) k = 2;
+  if (k > sms / 4) k = (sms / 4) & ~1;
+  return k;
+}
 
 void fill_layout(const moe_problem* pr, moe_tables_layout* L) {
   const int64_t E = pr->E;
@@ -450,6 +490,66 @@ moe_status moe_experts_forward(const moe_problem* prob, const void* hidden,
   const int T = prob->T, H = prob->H, F = prob->F, E = prob->E, k = prob->top_k;
 
   MOE_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int32_t), st));
+
+  // shared expert (a dense SwiGLU MLP on all tokens, added in the unpermute).
+  // Where the routed experts hold few rows each (at most 64 on average, the
+  // single-CTA weight-row tiling) their GEMMs are bound by weight bytes while
+  // the shared MLP is compute-bound, so it runs on its own stream and a few
+  // SMs beside them, joined before the unpermute: Kimi-K2 (T 512, 384
+  // experts) 5.14 vs 5.28 ms per layer. With more rows per expert the routed
+  // GEMMs need all SMs (DeepSeek-V3 prefill, 128 rows per expert: 4.75 with
+  // 16 SMs given away, 4.72 serial), and the shared expert runs after them.
+  const float* addend = nullptr;
+  cudaEvent_t join = nullptr;
+  int routed_ctas = 0;
+  if (prob->F_shared > 0) {
+    moe::GemmLaunch d;
+    d.rows = T;
+    d.E = 1;
+    d.status = status;
+    d.mode = moe::kModeSwiglu;
+    d.N = 2 * prob->F_shared;
+    d.K = H;
+    d.A = hidden;
+    d.B = ws_gate_up;
+    d.C = base + w.hs;
+    const bool beside = static_cast<int64_t>(T) * k <= 64LL * E;
+    cudaStream_t side = beside ? side_stream() : nullptr;
+    cudaStream_t sst = st;
+    cudaEvent_t fork = nullptr;
+    if (side != nullptr && cudaEventCreateWithFlags(&fork, cudaEventDisableTiming) == cudaSuccess) {
+      if (cudaEventCreateWithFlags(&join, cudaEventDisableTiming) != cudaSuccess) {
+        cudaEventDestroy(fork);
+        fork = join = nullptr;
+        cudaGetLastError();
+      }
+    } else {
+      fork = nullptr;
+      cudaGetLastError();
+    }
+    if (fork != nullptr) {
+      const int sms = moe::device_sm_count();
+      d.max_ctas = shared_sms(prob, sms);
+      routed_ctas = sms - d.max_ctas;
+      sst = side;
+      MOE_CUDA_TRY(cudaEventRecord(fork, st));
+      MOE_CUDA_TRY(cudaStreamWaitEvent(side, fork, 0));
+      cudaEventDestroy(fork);
+    }
+    MOE_CUDA_TRY(moe::launch_grouped_gemm(d, sst));
+    d.mode = moe::kModeStore;
+    d.N = H;
+    d.K = prob->F_shared;
+    d.A = base + w.hs;
+    d.B = ws_down;
+    d.C = base + w.ys;
+    d.out_f32 = 1;
+    MOE_CUDA_TRY(moe::launch_grouped_gemm(d, sst));
+    if (join != nullptr) MOE_CUDA_TRY(cudaEventRecord(join, side));
+    addend = reinterpret_cast<const float*>(base + w.ys);
+    g_last_launches += 2;
+  }
+
   // a2 + a3
   MOE_CUDA_TRY(moe::launch_tables(topk_ids, L.P, E, prob->padding_M, L.M_blk,
                                   tables + L.group_sizes, tables + L.group_offsets,
@@ -467,6 +567,7 @@ moe_status moe_experts_forward(const moe_problem* prob, const void* hidden,
   g.idx_for_bx = tables + L.group_idx_for_bx;
   g.M_blk = L.M_blk;
   g.status = status;
+  g.max_ctas = routed_ctas;
   // a4 + a5: gate+up with the SwiGLU (+ FP8 1x128) epilogue
   g.mode = prob->down_fp8 ? moe::kModeSwigluFp8 : moe::kModeSwiglu;
   g.N = 2 * F;
@@ -513,30 +614,9 @@ moe_status moe_experts_forward(const moe_problem* prob, const void* hidden,
   MOE_CUDA_TRY(moe::launch_grouped_gemm(g, st));
   g_last_launches += 2;
 
-  // shared expert: a dense SwiGLU MLP on all tokens, added in the unpermute
-  const float* addend = nullptr;
-  if (prob->F_shared > 0) {
-    moe::GemmLaunch d;
-    d.rows = T;
-    d.E = 1;
-    d.status = status;
-    d.mode = moe::kModeSwiglu;
-    d.N = 2 * prob->F_shared;
-    d.K = H;
-    d.A = hidden;
-    d.B = ws_gate_up;
-    d.C = base + w.hs;
-    MOE_CUDA_TRY(moe::launch_grouped_gemm(d, st));
-    d.mode = moe::kModeStore;
-    d.N = H;
-    d.K = prob->F_shared;
-    d.A = base + w.hs;
-    d.B = ws_down;
-    d.C = base + w.ys;
-    d.out_f32 = 1;
-    MOE_CUDA_TRY(moe::launch_grouped_gemm(d, st));
-    addend = reinterpret_cast<const float*>(base + w.ys);
-    g_last_launches += 2;
+  if (join != nullptr) {
+    MOE_CUDA_TRY(cudaStreamWaitEvent(st, join, 0));
+    cudaEventDestroy(join);
   }
   // a7
   if (f16e)

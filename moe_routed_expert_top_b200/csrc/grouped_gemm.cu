@@ -626,7 +626,8 @@ static cudaError_t run_gemm(const GemmLaunch& L, cudaStream_t stream) {
   const int NB = out_n / Cfg::OUT_COLS;
   const long long mblocks_ub = grouped ? static_cast<long long>(L.M_blk) : (L.rows + 127) / 128;
   const long long tiles_ub = mblocks_ub * NB;
-  const int sms = device_sm_count();
+  int sms = device_sm_count();
+  if (L.max_ctas > 0 && L.max_ctas < sms) sms = L.max_ctas;
   const int grid = static_cast<int>(tiles_ub < sms ? (tiles_ub > 0 ? tiles_ub : 1) : sms);
   grouped_gemm_kernel<kMode, BN><<<grid, 192, Cfg::SMEM_BYTES, stream>>>(tmA, tmB, p);
   return cudaGetLastError();

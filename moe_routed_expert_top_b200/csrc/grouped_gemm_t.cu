@@ -763,7 +763,8 @@ cudaError_t run_t(const GemmLaunch& L, cudaStream_t stream) {
   const long long chunks_ub = grouped ? (static_cast<long long>(L.rows) + TN - 1) / TN + E
                                       : (static_cast<long long>(L.rows) + TN - 1) / TN;
   const long long tiles_ub = chunks_ub * WB;
-  const int sms = device_sm_count();
+  int sms = device_sm_count();
+  if (L.max_ctas > 0 && L.max_ctas < sms) sms = L.max_ctas;
   const int grid = static_cast<int>(tiles_ub < sms ? (tiles_ub > 0 ? tiles_ub : 1) : sms);
   grouped_gemm_t_kernel<kMode, TN><<<grid, Cfg::kThreads, Cfg::SMEM_BYTES, stream>>>(
       tmW, tmX[0], tmX[1], tmX[2], tmX[3], p);

@@ -655,7 +655,8 @@ cudaError_t run_pair(const GemmLaunch& L, cudaStream_t stream) {
   const long long chunks_ub = grouped ? (static_cast<long long>(L.rows) + TN - 1) / TN + E
                                       : (static_cast<long long>(L.rows) + TN - 1) / TN;
   const long long pairs_ub = chunks_ub * WB;
-  const int max_pairs = max_pairs_cache[dev];
+  int max_pairs = max_pairs_cache[dev];
+  if (L.max_ctas > 0 && L.max_ctas / 2 < max_pairs) max_pairs = L.max_ctas / 2 > 0 ? L.max_ctas / 2 : 1;
   const int pairs = static_cast<int>(pairs_ub < max_pairs ? (pairs_ub > 0 ? pairs_ub : 1) : max_pairs);
   grouped_gemm_pair_kernel<kMode, TN, kGather><<<2 * pairs, kThreads, Cfg::SMEM_BYTES, stream>>>(
       tmW, tmX[0], tmX[1], tmX[2], tmX[3], p);

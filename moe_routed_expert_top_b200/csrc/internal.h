@@ -58,6 +58,9 @@ struct GemmLaunch {
   int weighted = 0;
   const float* row_weights = nullptr;
   float row_scale = 1.0f;
+  // at most this many CTAs (0 = one per SM): leaves SMs to a kernel that runs
+  // beside this one on another stream
+  int max_ctas = 0;
 };
 
 // Tiling of the grouped GEMM: token-row tiles (grouped_gemm.cu), weight-row
