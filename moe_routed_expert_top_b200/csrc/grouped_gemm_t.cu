@@ -88,8 +88,9 @@ struct TCfg {
   // (weighted store)
   static constexpr int STAGE_OUT_BYTES = 32 * 128 * 4 + 2 * TN * 4;
   // FP8: a scale warp (warp 6) prepares each tile's sa * sw products one tile
-  // ahead in a ring of two slots of TN x MAX_KBS fp32
-  static constexpr int kThreads = kFp8 ? 224 : 192;
+  // ahead in a ring of two slots of TN x MAX_KBS fp32, and a second MMA issuer
+  // (warp 7) takes every other K-block
+  static constexpr int kThreads = kFp8 ? 256 : 192;
   static constexpr int MAX_KBS = 16;                    // FP8: K <= 2048
   static constexpr int SA_SLOT = TN * MAX_KBS;          // floats per slot
   static constexpr int SA_BYTES = kFp8 ? 2 * SA_SLOT * 4 : 0;
@@ -292,7 +293,7 @@ __global__ void __launch_bounds__(TCfg<kMode, TN>::kThreads, 1)
       mbar_init(tfull0 + 8 * a, 1);
       mbar_init(tempty0 + 8 * a, 4);
     }
-    mbar_init(drain_bar, 1);
+    mbar_init(drain_bar, Cfg::kFp8 ? 2 : 1);  // one commit per MMA issuer
     if constexpr (Cfg::kFp8) {
       for (int i = 0; i < 2; ++i) {
         mbar_init(scl_full0 + 8 * i, 1);
@@ -406,9 +407,14 @@ __global__ void __launch_bounds__(TCfg<kMode, TN>::kThreads, 1)
         }
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || (Cfg::kFp8 && warp == 7)) {
+    // ------------------------------------------------------------ MMA issuer(s)
     if (lane == 0) {
+      // FP8: two issuers (warps 1 and 7) take the K-blocks of even and odd
+      // running index; each K-block has its own TMEM buffer and commit, so
+      // while one thread waits on the tensor pipe the other prepares the next
+      const int issuer = warp == 1 ? 0 : 1;
+      int nk = 0;  // running K-block index over the CTA's tiles
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -422,22 +428,24 @@ __global__ void __launch_bounds__(TCfg<kMode, TN>::kThreads, 1)
         if constexpr (Cfg::kFp8) {
           // one TMEM buffer per 128-wide K-block: the epilogue scales and sums them
           const uint32_t idesc8 = idesc_e4m3_f32(128, nmma);
-          for (int kb = 0; kb < KB; ++kb) {
-            if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag, p.status) ||
-                !mbar_wait(full0 + 8 * stage, phase, abort_flag, p.status)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t d = tmem_base + static_cast<uint32_t>(acc * TN);
-            const uint64_t adesc = smem_desc_sw128(smem_u32(sA + stage * Cfg::A_BYTES));
-            const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + stage * Cfg::B_BYTES));
+          for (int kb = 0; kb < KB; ++kb, ++nk) {
+            if ((nk & 1) == issuer) {
+              if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag, p.status) ||
+                  !mbar_wait(full0 + 8 * stage, phase, abort_flag, p.status)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t d = tmem_base + static_cast<uint32_t>(acc * TN);
+              const uint64_t adesc = smem_desc_sw128(smem_u32(sA + stage * Cfg::A_BYTES));
+              const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + stage * Cfg::B_BYTES));
 #pragma unroll
-            for (int k = 0; k < Cfg::K_STEPS; ++k)
-              mma_fp8(d, adesc + 2 * k, bdesc + 2 * k, idesc8, k != 0 ? 1u : 0u);
-            // one commit per K-block: the epilogue, which waits for this
-            // buffer anyway, releases the shared-memory stage when it lands
-            mma_commit(tfull0 + 8 * acc);
+              for (int k = 0; k < Cfg::K_STEPS; ++k)
+                mma_fp8(d, adesc + 2 * k, bdesc + 2 * k, idesc8, k != 0 ? 1u : 0u);
+              // one commit per K-block: the epilogue, which waits for this
+              // buffer anyway, releases the shared-memory stage when it lands
+              mma_commit(tfull0 + 8 * acc);
+            }
             if (++stage == STAGES) {
               stage = 0;
               phase ^= 1u;
