@@ -172,6 +172,93 @@ __global__ void __launch_bounds__(128) unpermute_f16e_kernel(
                                                      pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
 }
 
+// The same for k <= 8 as a persistent grid (8 blocks per SM) that walks its
+// (token, 128-column block) items in order and loads the next item's row
+// indices and weights while the current item's rows are in flight, so the
+// two dependent loads of an item (indices, then rows) do not add up. Same
+// arithmetic in the same order: results are identical.
+template <bool kAddend>
+__global__ void __launch_bounds__(128, 8) unpermute_f16e_pipe_kernel(
+    const uint4* __restrict__ y16, const int8_t* __restrict__ y_exp,
+    const int32_t* __restrict__ row_of_pair, const float* __restrict__ w, int k, int P, int H8,
+    float scale, const float4* __restrict__ addend, uint4* __restrict__ out, int cblocks,
+    long long items) {
+  const int HB = H8 / 16;
+  int nrows[8];
+  float nwts[8];
+  auto load_idx = [&](long long item) {
+    const int64_t pbase = (item / cblocks) * k;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const bool in = j < k;
+      const int r = in ? __ldg(row_of_pair + pbase + j) : -1;
+      nrows[j] = (r >= 0 && r < P) ? r : -1;
+      nwts[j] = in ? __ldg(w + pbase + j) : 0.0f;
+    }
+  };
+  long long item = blockIdx.x;
+  if (item < items) load_idx(item);
+  for (; item < items; item += gridDim.x) {
+    int rows[8];
+    float wts[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      rows[j] = nrows[j];
+      wts[j] = nwts[j];
+    }
+    const int64_t t = item / cblocks;
+    const int c = static_cast<int>(item - t * cblocks) * blockDim.x + threadIdx.x;
+    const bool col = c < H8;
+    uint4 va[8];
+    int ex[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (col && rows[j] >= 0) {
+        va[j] = __ldg(y16 + static_cast<int64_t>(rows[j]) * H8 + c);
+        ex[j] = __ldg(y_exp + static_cast<int64_t>(rows[j]) * HB + (c >> 4));
+      } else {
+        va[j] = make_uint4(0u, 0u, 0u, 0u);
+        ex[j] = 0;
+      }
+    }
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+    if (kAddend && col) {
+      const float4* ad = addend + (t * H8 + c) * 2;
+      a = __ldg(ad);
+      b = __ldg(ad + 1);
+    }
+    if (item + gridDim.x < items) load_idx(item + gridDim.x);
+    if (!col) continue;
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (j >= k) break;
+      if (rows[j] < 0) continue;
+      const float s2 = f16e_pow2(ex[j]);
+      const uint32_t wd[4] = {va[j].x, va[j].y, va[j].z, va[j].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wd[q]));
+        acc[2 * q] = fmaf(wts[j], f.x * s2, acc[2 * q]);
+        acc[2 * q + 1] = fmaf(wts[j], f.y * s2, acc[2 * q + 1]);
+      }
+    }
+    float v[8];
+    if constexpr (kAddend) {
+      const float add[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = fmaf(scale, acc[i], add[i]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = scale * acc[i];
+    }
+    out[t * H8 + c] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                 pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+  }
+}
+
 cudaError_t launch_unpermute_f16e(const void* y16, const int8_t* y_exp, const int32_t* row_of_pair,
                                   const float* weights, int T, int k, int H, float scale,
                                   const float* addend, void* out, cudaStream_t stream) {
@@ -179,6 +266,20 @@ cudaError_t launch_unpermute_f16e(const void* y16, const int8_t* y_exp, const in
   const int H8 = H / 8;
   const int cblocks = (H8 + 127) / 128;
   const long long blocks = static_cast<long long>(T) * cblocks;
+  if (k <= 8) {
+    const long long cap = static_cast<long long>(device_sm_count()) * 8;
+    const unsigned grid = static_cast<unsigned>(blocks < cap ? blocks : cap);
+    const float4* ad = reinterpret_cast<const float4*>(addend);
+    if (addend != nullptr)
+      unpermute_f16e_pipe_kernel<true><<<grid, 128, 0, stream>>>(
+          static_cast<const uint4*>(y16), y_exp, row_of_pair, weights, k, T * k, H8, scale, ad,
+          static_cast<uint4*>(out), cblocks, blocks);
+    else
+      unpermute_f16e_pipe_kernel<false><<<grid, 128, 0, stream>>>(
+          static_cast<const uint4*>(y16), y_exp, row_of_pair, weights, k, T * k, H8, scale, ad,
+          static_cast<uint4*>(out), cblocks, blocks);
+    return cudaGetLastError();
+  }
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   unpermute_f16e_kernel<<<static_cast<unsigned>(blocks), 128, 0, stream>>>(
       static_cast<const uint4*>(y16), y_exp, row_of_pair, weights, k, T * k, H8, scale,
