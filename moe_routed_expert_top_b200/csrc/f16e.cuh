@@ -29,17 +29,18 @@ __device__ __forceinline__ float f16e_pow2(int x) {
   return __uint_as_float(static_cast<uint32_t>(x + 127) << 23);
 }
 
-// Encodes four rows' blocks at once (the four row passes of a 32-row slab).
-// Each row's 128-column block is spread over 16 consecutive lanes of a half
-// warp, 8 columns each (v[q]: this lane's 8 values of pass q); every lane of
-// the warp must call this. Returns each block's exponent (the same in its 16
-// lanes) and this lane's 8 fp16 codes per pass. The four half-warp reductions
-// are interleaved so that their shuffle latencies overlap.
-__device__ __forceinline__ void f16e_encode8x4(const float (&v)[4][8], uint4 (&out)[4],
-                                               int (&e)[4]) {
-  float amax[4];
+// Encodes NP rows' blocks at once (the NP row passes of a slab). Each row's
+// 128-column block is spread over 16 consecutive lanes of a half warp, 8
+// columns each (v[q]: this lane's 8 values of pass q); every lane of the warp
+// must call this. Returns each block's exponent (the same in its 16 lanes)
+// and this lane's 8 fp16 codes per pass. The NP half-warp reductions are
+// interleaved so that their shuffle latencies overlap.
+template <int NP>
+__device__ __forceinline__ void f16e_encode8xn(const float (&v)[NP][8], uint4 (&out)[NP],
+                                               int (&e)[NP]) {
+  float amax[NP];
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
+  for (int q = 0; q < NP; ++q) {
     amax[q] = 0.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) amax[q] = fmaxf(amax[q], fabsf(v[q][i]));
@@ -47,10 +48,11 @@ __device__ __forceinline__ void f16e_encode8x4(const float (&v)[4][8], uint4 (&o
 #pragma unroll
   for (int off = 8; off > 0; off >>= 1) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) amax[q] = fmaxf(amax[q], __shfl_xor_sync(0xffffffffu, amax[q], off));
+    for (int q = 0; q < NP; ++q)
+      amax[q] = fmaxf(amax[q], __shfl_xor_sync(0xffffffffu, amax[q], off));
   }
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
+  for (int q = 0; q < NP; ++q) {
     e[q] = f16e_exponent(amax[q]);
     const float s = f16e_pow2(-e[q]);
     uint32_t w[4];

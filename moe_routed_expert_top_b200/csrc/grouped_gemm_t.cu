@@ -180,7 +180,7 @@ __device__ __forceinline__ void store_rows(const TParams& p, const float* sOut, 
     }
     uint4 pk[4];
     int e[4];
-    f16e_encode8x4(v, pk, e);
+    f16e_encode8xn<4>(v, pk, e);
 #pragma unroll
     for (int pass = 0; pass < 4; ++pass) {
       const int i = pass * 8 + (et >> 4);

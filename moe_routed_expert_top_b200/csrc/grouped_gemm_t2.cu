@@ -82,9 +82,9 @@ struct PCfg {
   static constexpr int STAGES = pmin(8, (200 * 1024) / STAGE_BYTES);
   static constexpr int NUM_ACC = 2;
   static constexpr int TMEM_COLS = 2 * TN;
-  // 32 token rows x 128 fp32, then the tile's row destinations and factors
-  // (weighted store)
-  static constexpr int STAGE_OUT_BYTES = 32 * 128 * 4 + 2 * TN * 4;
+  // 32 token rows x 128 fp32 (16 per epilogue group), then each group's copy
+  // of the tile's row destinations and factors (weighted store)
+  static constexpr int STAGE_OUT_BYTES = 32 * 128 * 4 + 4 * TN * 4;
   static constexpr int NUM_BARS = 2 * STAGES + 2 * NUM_ACC + 1;
   static constexpr int MAX_E = 1024;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STAGE_OUT_BYTES +
@@ -133,7 +133,13 @@ __device__ __forceinline__ int half_box(int half) {  // smallest of 16/32/64/128
   return half <= 16 ? 0 : half <= 32 ? 1 : half <= 64 ? 2 : 3;
 }
 
-__device__ __forceinline__ void pepi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Named barrier of epilogue group g (its 128 threads).
+__device__ __forceinline__ void pgroup_bar(int g) {
+  if (g == 0)
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+  else
+    asm volatile("bar.sync 2, 128;" ::: "memory");
+}
 
 __device__ __forceinline__ float psilu(float g) { return g / (1.0f + expf(-g)); }
 
@@ -144,7 +150,7 @@ __device__ __forceinline__ void pair_commit(uint32_t bar) {
 }
 
 // Threads per CTA: producer warp, MMA warp, 4 epilogue warps.
-constexpr int kPairThreads = 192;
+constexpr int kPairThreads = 320;  // TMA, MMA, two groups of 4 epilogue warps
 
 template <int kMode, int TN, bool kGather>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
@@ -164,8 +170,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * Cfg::A_BYTES;
   float* sOut = reinterpret_cast<float*>(sB + STAGES * Cfg::B_BYTES);
-  int* sDst = reinterpret_cast<int*>(sOut + 32 * 128);  // weighted store: the tile's row info
-  float* sFac = reinterpret_cast<float*>(sDst + TN);
+  int* sDst = reinterpret_cast<int*>(sOut + 32 * 128);  // weighted store: [2][TN] row info
+  float* sFac = reinterpret_cast<float*>(sDst + 2 * TN);   // [2][TN]
   uint64_t* bars =
       reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sOut) + Cfg::STAGE_OUT_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cfg::NUM_BARS);
@@ -195,7 +201,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     }
     for (int a = 0; a < NUM_ACC; ++a) {
       mbar_init(tfull0 + 8 * a, 1);
-      mbar_init(tempty0 + 8 * a, 8);  // 4 epilogue warps in each CTA of the pair
+      mbar_init(tempty0 + 8 * a, 16);  // 8 epilogue warps in each CTA of the pair
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -412,10 +418,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
+    // Two groups of four warps (2-5 and 6-9). In each 32-token slab of a tile,
+    // group g takes tokens 16g .. 16g+15: its own TMEM columns, its own 16 rows
+    // of sOut and its own named barrier, so one group's stores and barrier
+    // waits overlap the other's TMEM loads. Warp w reads TMEM lanes
+    // 32*(w%4) .. +31 (its weight rows).
+    const int grp = (warp - 2) >> 2;
     const int q = warp & 3;
     const int r = q * 32 + lane;
-    const int et = threadIdx.x - 64;
+    const int et = threadIdx.x - 64 - 128 * grp;  // 0..127 within the group
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    float* gOut = sOut + grp * 16 * 128;
+    int* gDst = sDst + grp * TN;
+    float* gFac = sFac + grp * TN;
     int acc = 0;
     uint32_t acc_phase = 0;
     int ecur = 0;
@@ -424,41 +439,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       if (!p_decode(p, cpre, soff, WB, TN, t, ecur, ti)) continue;
       if (kMode == kPStore && p.weighted) {
         // the tile's row destinations (flat pair index, -1 = none) and factors,
-        // loaded while its MMAs run; read after the first chunk's barrier
+        // loaded while its MMAs run; read after the first slab's barrier
         for (int i = et; i < ti.nt; i += 128) {
           const int pr = __ldg(p.pair_of_row + ti.m0 + i);
-          sDst[i] = pr;
-          sFac[i] = pr >= 0 ? p.row_scale * __ldg(p.row_w + pr) : 0.0f;
+          gDst[i] = pr;
+          gFac[i] = pr >= 0 ? p.row_scale * __ldg(p.row_w + pr) : 0.0f;
         }
       }
       if (!mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, p.status)) *epi_abort = 1;
-      pepi_bar();
+      pgroup_bar(grp);
       if (*epi_abort) break;
       tc_fence_after();
-      const uint32_t tb = lane_base + static_cast<uint32_t>(acc * TN);
+      const uint32_t tb = lane_base + static_cast<uint32_t>(acc * TN + 16 * grp);
       const int col0 = ti.wb * Cfg::PAIR_COLS + static_cast<int>(rank) * Cfg::CTA_COLS;
-      uint32_t v[32], vn[32];
-      tmem_ld32(tb, v);
+      uint32_t v[16], vn[16];
+      tmem_ld16(tb, v);
       tmem_ld_wait();
       for (int j0 = 0; j0 < ti.nt; j0 += 32) {
         const bool more = j0 + 32 < ti.nt;
-        if (more) tmem_ld32(tb + j0 + 32, vn);
+        if (more) tmem_ld16(tb + j0 + 32, vn);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) sOut[i * 128 + r] = __uint_as_float(v[i]);
-        const int rows = pmin(32, ti.nt - j0);
-        pepi_bar();
+        for (int i = 0; i < 16; ++i) gOut[i * 128 + r] = __uint_as_float(v[i]);
+        const int jg = j0 + 16 * grp;  // the group's first token of this slab
+        const int rows = pmin(16, ti.nt - jg);  // may be <= 0: nothing to store
+        pgroup_bar(grp);
         if constexpr (kMode == kPStore) {
           if (p.out_f32) {
 #pragma unroll
-            for (int pass = 0; pass < 8; ++pass) {
+            for (int pass = 0; pass < 4; ++pass) {
               const int i = pass * 4 + (et >> 5);
               const int c4 = et & 31;
               if (i < rows) {
-                float4 val = reinterpret_cast<const float4*>(sOut + i * 128)[c4];
-                int drow = ti.m0 + j0 + i;
+                float4 val = reinterpret_cast<const float4*>(gOut + i * 128)[c4];
+                int drow = ti.m0 + jg + i;
                 if (p.weighted) {
-                  drow = sDst[j0 + i];
-                  const float f = sFac[j0 + i];
+                  drow = gDst[jg + i];
+                  const float f = gFac[jg + i];
                   if (drow < 0) continue;
                   val = make_float4(val.x * f, val.y * f, val.z * f, val.w * f);
                 }
@@ -470,23 +486,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             // f16e: a row's 128 columns are this CTA's output block, held by 16
             // lanes of a half warp (8 columns each); every lane encodes
             const int c8 = et & 15;
-            float fv[4][8];
+            float fv[2][8];
 #pragma unroll
-            for (int pass = 0; pass < 4; ++pass) {
+            for (int pass = 0; pass < 2; ++pass) {
               const float4* src =
-                  reinterpret_cast<const float4*>(sOut + (pass * 8 + (et >> 4)) * 128 + c8 * 8);
+                  reinterpret_cast<const float4*>(gOut + (pass * 8 + (et >> 4)) * 128 + c8 * 8);
               const float4 a = src[0], b = src[1];
               fv[pass][0] = a.x; fv[pass][1] = a.y; fv[pass][2] = a.z; fv[pass][3] = a.w;
               fv[pass][4] = b.x; fv[pass][5] = b.y; fv[pass][6] = b.z; fv[pass][7] = b.w;
             }
-            uint4 pk[4];
-            int e[4];
-            f16e_encode8x4(fv, pk, e);
+            uint4 pk[2];
+            int e[2];
+            f16e_encode8xn<2>(fv, pk, e);
 #pragma unroll
-            for (int pass = 0; pass < 4; ++pass) {
+            for (int pass = 0; pass < 2; ++pass) {
               const int i = pass * 8 + (et >> 4);
               if (i < rows) {
-                const int64_t row = ti.m0 + j0 + i;
+                const int64_t row = ti.m0 + jg + i;
                 __half* dst = static_cast<__half*>(p.C) + row * p.ldc + col0;
                 reinterpret_cast<uint4*>(dst)[c8] = pk[pass];
                 if (c8 == 0)
@@ -495,16 +511,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             }
           } else {
 #pragma unroll
-            for (int pass = 0; pass < 4; ++pass) {
+            for (int pass = 0; pass < 2; ++pass) {
               const int i = pass * 8 + (et >> 4);
               const int c8 = et & 15;
               if (i < rows) {
-                const float* src = sOut + i * 128 + c8 * 8;
-                int drow = ti.m0 + j0 + i;
+                const float* src = gOut + i * 128 + c8 * 8;
+                int drow = ti.m0 + jg + i;
                 float f = 1.0f;
                 if (p.weighted) {
-                  drow = sDst[j0 + i];
-                  f = sFac[j0 + i];
+                  drow = gDst[jg + i];
+                  f = gFac[jg + i];
                   if (drow < 0) continue;
                 }
                 const uint4 val =
@@ -521,29 +537,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             }
           }
         } else {
+          // swiglu: gate = weight rows 0..63, up = rows 64..127 of this CTA's
+          // block; an h row = 64 bf16 = 8 x 16 B; 16 rows per pass
+          const int i = et >> 3;
+          const int c8 = et & 7;
+          if (i < rows) {
+            const float* g = gOut + i * 128 + c8 * 8;
+            const float* u = g + 64;
+            uint32_t pk[4];
 #pragma unroll
-          for (int pass = 0; pass < 2; ++pass) {
-            const int i = pass * 16 + (et >> 3);
-            const int c8 = et & 7;
-            if (i < rows) {
-              const float* g = sOut + i * 128 + c8 * 8;
-              const float* u = g + 64;
-              uint32_t pk[4];
-#pragma unroll
-              for (int k2 = 0; k2 < 4; ++k2)
-                pk[k2] = pack_bf16x2(psilu(g[2 * k2]) * u[2 * k2],
-                                     psilu(g[2 * k2 + 1]) * u[2 * k2 + 1]);
-              __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.C) +
-                                   static_cast<int64_t>(ti.m0 + j0 + i) * p.ldc + col0;
-              reinterpret_cast<uint4*>(dst)[c8] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            }
+            for (int k2 = 0; k2 < 4; ++k2)
+              pk[k2] = pack_bf16x2(psilu(g[2 * k2]) * u[2 * k2],
+                                   psilu(g[2 * k2 + 1]) * u[2 * k2 + 1]);
+            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.C) +
+                                 static_cast<int64_t>(ti.m0 + jg + i) * p.ldc + col0;
+            reinterpret_cast<uint4*>(dst)[c8] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
         }
-        pepi_bar();
+        pgroup_bar(grp);  // the group's rows of sOut are rewritten by its next slab
         if (more) {
           tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = vn[i];
+          for (int i = 0; i < 16; ++i) v[i] = vn[i];
         }
       }
       tc_fence_before();
