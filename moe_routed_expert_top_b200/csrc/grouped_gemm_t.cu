@@ -88,9 +88,10 @@ struct TCfg {
   // (weighted store)
   static constexpr int STAGE_OUT_BYTES = 32 * 128 * 4 + 2 * TN * 4;
   // FP8: a scale warp (warp 6) prepares each tile's sa * sw products one tile
-  // ahead in a ring of two slots of TN x MAX_KBS fp32, and a second MMA issuer
-  // (warp 7) takes every other K-block
-  static constexpr int kThreads = kFp8 ? 256 : 192;
+  // ahead in a ring of two slots of TN x MAX_KBS fp32, a second MMA issuer
+  // (warp 7) takes every other K-block, and a second epilogue group (warps
+  // 8-11) takes the tile's token columns 32..63
+  static constexpr int kThreads = kFp8 ? 384 : 192;
   static constexpr int MAX_KBS = 16;                    // FP8: K <= 2048
   static constexpr int SA_SLOT = TN * MAX_KBS;          // floats per slot
   static constexpr int SA_BYTES = kFp8 ? 2 * SA_SLOT * 4 : 0;
@@ -143,6 +144,9 @@ __device__ __forceinline__ int xbox_for(int n) {  // smallest box (32/64/128/256
 }
 
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// FP8: the second epilogue group's barrier, and both groups' (256 threads)
+__device__ __forceinline__ void epi_bar_g1() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+__device__ __forceinline__ void epi_bar_all() { asm volatile("bar.sync 3, 256;" ::: "memory"); }
 
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
 
@@ -291,7 +295,7 @@ __global__ void __launch_bounds__(TCfg<kMode, TN>::kThreads, 1)
     }
     for (int a = 0; a < NUM_ACC; ++a) {
       mbar_init(tfull0 + 8 * a, 1);
-      mbar_init(tempty0 + 8 * a, 4);
+      mbar_init(tempty0 + 8 * a, Cfg::kFp8 ? 8 : 4);  // epilogue warps
     }
     mbar_init(drain_bar, Cfg::kFp8 ? 2 : 1);  // one commit per MMA issuer
     if constexpr (Cfg::kFp8) {
@@ -544,7 +548,9 @@ __global__ void __launch_bounds__(TCfg<kMode, TN>::kThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
     const int r = q * 32 + lane;  // weight row of this thread's TMEM lane
-    const int et = threadIdx.x - 64;  // 0..127 within the epilogue warps
+    // FP8: two groups, warps 2-5 (token columns 0..31) and 8-11 (32..63)
+    const int grp = (Cfg::kFp8 && warp >= 8) ? 1 : 0;
+    const int et = threadIdx.x - (grp ? 256 : 64);  // 0..127 within the group
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -555,17 +561,20 @@ __global__ void __launch_bounds__(TCfg<kMode, TN>::kThreads, 1)
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
       TTile ti;
       if (!t_decode(p, cpre, soff, WB, TN, t, ecur, ti)) continue;
-      if (kMode != kTSwiglu && p.weighted) stage_row_info(p, et, ti.nt, ti.m0, sDst, sFac);
+      if (kMode != kTSwiglu && p.weighted && grp == 0)
+        stage_row_info(p, et, ti.nt, ti.m0, sDst, sFac);
       if constexpr (Cfg::kFp8) {
         // y[t, w] = sum_kb sw[e, wb, kb] * sa[t, kb] * (Wq_kb Xq_kb^T)[w, t], with
-        // the tile's products sw * sa prepared by the scale warp in slot sslot
+        // the tile's products sw * sa prepared by the scale warp in slot sslot;
+        // group grp holds token columns 32*grp .. 32*grp+31
         const float* sS = sSa + sslot * Cfg::SA_SLOT;
         if (!mbar_wait(scl_full0 + 8 * sslot, sphase, abort_flag, p.status)) *epi_abort = 1;
-        epi_bar();  // every epilogue warp arrives here whether its wait succeeded or not
+        epi_bar_all();  // both groups arrive here whether their waits succeeded or not
         if (*epi_abort) break;
-        float accv[TN];
+        const bool mine = grp * 32 < ti.nt;  // uniform across the group
+        float accv[32];
 #pragma unroll
-        for (int i = 0; i < TN; ++i) accv[i] = 0.0f;
+        for (int i = 0; i < 32; ++i) accv[i] = 0.0f;
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, p.status)) {
@@ -573,28 +582,22 @@ __global__ void __launch_bounds__(TCfg<kMode, TN>::kThreads, 1)
             break;
           }
           // this K-block's MMAs have completed: its shared-memory stage is free
-          if (et == 0) mbar_arrive(empty0 + 8 * stage);
+          if (grp == 0 && et == 0) mbar_arrive(empty0 + 8 * stage);
           if (++stage == STAGES) stage = 0;
           tc_fence_after();
-          const uint32_t tbk = lane_base + static_cast<uint32_t>(acc * TN);
-          const float4* s4 = reinterpret_cast<const float4*>(sS + kb * TN);
-          uint32_t v[TN / 32][32];
+          if (mine) {
+            const uint32_t tbk = lane_base + static_cast<uint32_t>(acc * TN + grp * 32);
+            const float4* s4 = reinterpret_cast<const float4*>(sS + kb * TN + grp * 32);
+            uint32_t v[32];
+            tmem_ld32(tbk, v);
+            tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < TN / 32; ++c)
-            if (c * 32 < ti.nt) tmem_ld32(tbk + c * 32, v[c]);  // uniform across the warp
-          tmem_ld_wait();
-#pragma unroll
-          for (int c = 0; c < TN / 32; ++c) {
-            if (c * 32 < ti.nt) {
-#pragma unroll
-              for (int i4 = 0; i4 < 8; ++i4) {
-                const float4 s = s4[c * 8 + i4];
-                const int col = c * 32 + i4 * 4;
-                accv[col + 0] = fmaf(s.x, __uint_as_float(v[c][i4 * 4 + 0]), accv[col + 0]);
-                accv[col + 1] = fmaf(s.y, __uint_as_float(v[c][i4 * 4 + 1]), accv[col + 1]);
-                accv[col + 2] = fmaf(s.z, __uint_as_float(v[c][i4 * 4 + 2]), accv[col + 2]);
-                accv[col + 3] = fmaf(s.w, __uint_as_float(v[c][i4 * 4 + 3]), accv[col + 3]);
-              }
+            for (int i4 = 0; i4 < 8; ++i4) {
+              const float4 sc = s4[i4];
+              accv[i4 * 4 + 0] = fmaf(sc.x, __uint_as_float(v[i4 * 4 + 0]), accv[i4 * 4 + 0]);
+              accv[i4 * 4 + 1] = fmaf(sc.y, __uint_as_float(v[i4 * 4 + 1]), accv[i4 * 4 + 1]);
+              accv[i4 * 4 + 2] = fmaf(sc.z, __uint_as_float(v[i4 * 4 + 2]), accv[i4 * 4 + 2]);
+              accv[i4 * 4 + 3] = fmaf(sc.w, __uint_as_float(v[i4 * 4 + 3]), accv[i4 * 4 + 3]);
             }
           }
           tc_fence_before();
@@ -606,25 +609,25 @@ __global__ void __launch_bounds__(TCfg<kMode, TN>::kThreads, 1)
           }
         }
         if (!ok) *epi_abort = 1;
-        epi_bar();
+        epi_bar_all();
         if (*epi_abort) break;
         // every epilogue thread is done with the slot: the scale warp may refill it
-        if (et == 0) mbar_arrive(scl_empty0 + 8 * sslot);
+        if (grp == 0 && et == 0) mbar_arrive(scl_empty0 + 8 * sslot);
         if (++sslot == 2) {
           sslot = 0;
           sphase ^= 1u;
         }
+        // the groups store their 32 token rows in turn through sOut
+        if (grp == 1) epi_bar_all();
+        if (mine) {
 #pragma unroll
-        for (int c = 0; c < TN / 32; ++c) {
-          if (c * 32 < ti.nt) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) sOut[i * 128 + r] = accv[c * 32 + i];
-            epi_bar();
-            store_rows(p, sOut, et, tmin(32, ti.nt - c * 32), ti.m0 + c * 32, ti.wb * 128,
-                       sDst + c * 32, sFac + c * 32);
-            epi_bar();
-          }
+          for (int i = 0; i < 32; ++i) sOut[i * 128 + r] = accv[i];
+          if (grp == 0) epi_bar(); else epi_bar_g1();
+          store_rows(p, sOut, et, tmin(32, ti.nt - grp * 32), ti.m0 + grp * 32, ti.wb * 128,
+                     sDst + grp * 32, sFac + grp * 32);
         }
+        if (grp == 0) epi_bar_all();
+        epi_bar_all();  // sOut and the row info are rewritten for the next tile
         continue;
       }
       if (!mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, p.status)) *epi_abort = 1;
