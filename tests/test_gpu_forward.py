@@ -93,6 +93,10 @@ MID = [
                score_fn="sigmoid", routed_scaling_factor=2.5, F_shared=192, seed=22),
     get_config("tiny", name="mid_fp8", T=190, E=10, top_k=4, H=256, F=512, score_fn="sigmoid",
                routed_scaling_factor=2.5, down_fp8=True, seed=23),
+    # at most 64 rows per routed expert: the shared expert runs on the side
+    # stream beside the routed GEMMs (on a capped set of SMs)
+    get_config("tiny", name="mid_shared_beside", T=200, E=16, top_k=2, H=256, F=256,
+               score_fn="sigmoid", routed_scaling_factor=2.5, F_shared=384, seed=24),
 ]
 
 
@@ -175,6 +179,30 @@ def test_single_token_and_edge_group_sizes():
     hidden, ids, w, weights = _inputs(cfg, ids=ids)
     out, _ = _run(cfg, hidden, ids, w, weights)
     gu.assert_within_tol(gu.f64(out), _oracle(cfg, hidden, ids, w, weights), "edge sizes")
+
+
+def test_graph_replay_matches_eager():
+    """The forward captured as a CUDA graph (the side stream of the shared
+    expert becomes a fork and a join in the graph) and replayed gives the eager
+    call's output bit for bit."""
+    cfg = next(c for c in MID if c.name == "mid_shared_beside")
+    hidden, ids, w, weights = _inputs(cfg)
+    eager, layer = _run(cfg, hidden, ids, w, weights)
+    ids_d = torch.from_numpy(ids).cuda()
+    w_d = torch.from_numpy(w).cuda()
+    out = torch.empty_like(eager)
+    layer.forward(hidden, ids_d, w_d, out)  # workspace allocated before capture
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        layer.forward(hidden, ids_d, w_d, out)
+    out.zero_()
+    graph.replay()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    assert torch.equal(out.view(torch.int16), eager.view(torch.int16))
+    del graph
 
 
 def test_deterministic_repeat():

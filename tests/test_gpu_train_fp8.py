@@ -208,6 +208,44 @@ def test_full_size_sampled_blocks():
                 assert np.array_equal(sT[kb * 128:(kb + 1) * 128, bx].cpu().numpy(), bs[:, 0])
 
 
+def test_more_tiles_than_the_rows_table_holds():
+    """Dense x [20000037, 128]: 156251 128x128 tiles, more per persistent CTA
+    than the kernel's precomputed table of tile rows holds (512), so the last
+    tiles of every CTA take their rows from the tables as they go, and the
+    row and column offsets pass 2^31 bytes. Sampled rows and blocks, the
+    ragged last block among them, against the oracle."""
+    import moe_routed_expert_top_b200 as Mo
+    M, K = 20000037, 128
+    rng = np.random.default_rng(31)
+    M_blk = Mo.moe_dual_blocks(None, M)
+    assert M_blk == (M + 127) // 128
+    torch.manual_seed(31)
+    x = torch.randn(M, K, device="cuda", dtype=torch.bfloat16)
+    for per_block in (True, False):
+        q, s, qT, sT = _outputs(M, K, M_blk, per_block)
+        mode = Mo.MOE_TRANS_PER_BLOCK if per_block else Mo.MOE_TRANS_PER_TILE
+        Mo.moe_quant_dual(None, None, M, K, x, mode, q, s, qT, sT)
+        torch.cuda.synchronize()
+        rows = np.concatenate([rng.choice(M, 8, replace=False), [M - 1, M - 37, 19_500_000]])
+        ridx = torch.from_numpy(rows).cuda()
+        rq, rs = O.quant_1x128(x[ridx].float().cpu().numpy())
+        assert np.array_equal(q[ridx].cpu().numpy(), rq)
+        assert np.array_equal(s[ridx].cpu().numpy(), rs)
+        for bx in list(rng.integers(152_000, M_blk - 1, 4)) + [0, M_blk - 1]:
+            m0 = int(bx) * 128
+            n = min(128, M - m0)
+            blk = x[m0:m0 + n].float().cpu().numpy()
+            bq, bs = O.quant_transposed(blk, np.arange(n), 128, per_block)
+            got = qT[:, int(bx) * 128:(int(bx) + 1) * 128].cpu().numpy()
+            assert np.array_equal(got, bq)
+            if per_block:
+                assert sT[0, int(bx)].item() == bs[0, 0]
+            else:
+                assert np.array_equal(sT[:, int(bx)].cpu().numpy(), bs[:, 0])
+        del q, s, qT, sT
+        torch.cuda.empty_cache()
+
+
 def test_train_fp8_rejects():
     import moe_routed_expert_top_b200 as Mo
     x = torch.zeros(8, 128, dtype=torch.bfloat16, device="cuda")
