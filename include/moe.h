@@ -333,7 +333,13 @@ moe_status moe_quantize_weight_128x128(int32_t batch, int32_t N, int32_t K, cons
  *   [H, F_s] when F_shared > 0 (else NULL).
  * Needs prob->padding_M == 128. `workspace` (ws_bytes >= moe_workspace_bytes)
  * is caller-owned device memory; its first int32 is this call's device status
- * (zeroed by the call, then OR-ed with MOE_DEV_* flags). */
+ * (zeroed by the call, then OR-ed with MOE_DEV_* flags).
+ * Streams: everything is ordered on `stream`. When F_shared > 0 and the routed
+ * experts average at most 64 rows (T*k <= 64*E), the shared expert's two GEMMs
+ * run on a second, library-owned stream of the current device (created on first
+ * use, never destroyed), forked from `stream` by an event before them and joined
+ * back by an event before the unpermute; the routed GEMMs then use the other SMs.
+ * Under CUDA graph capture of `stream` the fork and join are graph edges. */
 moe_status moe_experts_forward(const moe_problem* prob, const void* hidden,
                                const int32_t* topk_ids, const float* topk_weights,
                                const void* w_gate_up, const void* w_down,
