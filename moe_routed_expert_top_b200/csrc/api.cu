@@ -76,6 +76,21 @@ cudaStream_t side_stream() {
   return streams[dev];
 }
 
+// An event released when the forward returns (also on its error paths);
+// destroying an event whose record and waits are enqueued is allowed.
+struct EventGuard {
+  cudaEvent_t e = nullptr;
+  bool create() {
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess) return true;
+    e = nullptr;
+    cudaGetLastError();
+    return false;
+  }
+  ~EventGuard() {
+    if (e != nullptr) cudaEventDestroy(e);
+  }
+};
+
 // SMs given to the shared expert while the routed GEMMs run on the others, so
 // that both finish at about the same time: the shared MLP is compute-bound
 // (its FLOPs at about 0.9 PFLOP/s, the dense rate its tiles reach on B200),
@@ -500,7 +515,8 @@ moe_status moe_experts_forward(const moe_problem* prob, const void* hidden,
   // GEMMs need all SMs (DeepSeek-V3 prefill, 128 rows per expert: 4.75 with
   // 16 SMs given away, 4.72 serial), and the shared expert runs after them.
   const float* addend = nullptr;
-  cudaEvent_t join = nullptr;
+  EventGuard fork, join;
+  bool beside = false;
   int routed_ctas = 0;
   if (prob->F_shared > 0) {
     moe::GemmLaunch d;
@@ -513,28 +529,16 @@ moe_status moe_experts_forward(const moe_problem* prob, const void* hidden,
     d.A = hidden;
     d.B = ws_gate_up;
     d.C = base + w.hs;
-    const bool beside = static_cast<int64_t>(T) * k <= 64LL * E;
-    cudaStream_t side = beside ? side_stream() : nullptr;
+    cudaStream_t side = static_cast<int64_t>(T) * k <= 64LL * E ? side_stream() : nullptr;
+    beside = side != nullptr && fork.create() && join.create();
     cudaStream_t sst = st;
-    cudaEvent_t fork = nullptr;
-    if (side != nullptr && cudaEventCreateWithFlags(&fork, cudaEventDisableTiming) == cudaSuccess) {
-      if (cudaEventCreateWithFlags(&join, cudaEventDisableTiming) != cudaSuccess) {
-        cudaEventDestroy(fork);
-        fork = join = nullptr;
-        cudaGetLastError();
-      }
-    } else {
-      fork = nullptr;
-      cudaGetLastError();
-    }
-    if (fork != nullptr) {
+    if (beside) {
       const int sms = moe::device_sm_count();
       d.max_ctas = shared_sms(prob, sms);
       routed_ctas = sms - d.max_ctas;
       sst = side;
-      MOE_CUDA_TRY(cudaEventRecord(fork, st));
-      MOE_CUDA_TRY(cudaStreamWaitEvent(side, fork, 0));
-      cudaEventDestroy(fork);
+      MOE_CUDA_TRY(cudaEventRecord(fork.e, st));
+      MOE_CUDA_TRY(cudaStreamWaitEvent(side, fork.e, 0));
     }
     MOE_CUDA_TRY(moe::launch_grouped_gemm(d, sst));
     d.mode = moe::kModeStore;
@@ -545,7 +549,7 @@ moe_status moe_experts_forward(const moe_problem* prob, const void* hidden,
     d.C = base + w.ys;
     d.out_f32 = 1;
     MOE_CUDA_TRY(moe::launch_grouped_gemm(d, sst));
-    if (join != nullptr) MOE_CUDA_TRY(cudaEventRecord(join, side));
+    if (beside) MOE_CUDA_TRY(cudaEventRecord(join.e, side));
     addend = reinterpret_cast<const float*>(base + w.ys);
     g_last_launches += 2;
   }
@@ -614,10 +618,7 @@ moe_status moe_experts_forward(const moe_problem* prob, const void* hidden,
   MOE_CUDA_TRY(moe::launch_grouped_gemm(g, st));
   g_last_launches += 2;
 
-  if (join != nullptr) {
-    MOE_CUDA_TRY(cudaStreamWaitEvent(st, join, 0));
-    cudaEventDestroy(join);
-  }
+  if (beside) MOE_CUDA_TRY(cudaStreamWaitEvent(st, join.e, 0));
   // a7
   if (f16e)
     MOE_CUDA_TRY(moe::launch_unpermute_f16e(y, y_exp, tables + L.row_of_pair, topk_weights, T, k,
