@@ -22,7 +22,9 @@
 //            r + 64 through shared memory (XTuner PR #2089, SiLU(gate)*up).
 // Warp roles and the bounded-wait/teardown protocol are those of
 // grouped_gemm.cu: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer,
-// warps 2-5 epilogue (TMEM lane = weight row), two TMEM accumulators.
+// warps 2-5 epilogue (TMEM lane = weight row), two TMEM accumulators. The FP8
+// mode adds a scale warp (6), a second MMA issuer (7) and a second epilogue
+// group (8-11), 384 threads.
 // The epilogue stages 32 token rows at a time in shared memory and writes
 // them row-major with 16-byte stores, masking rows past the tile's tokens.
 #include <cuda.h>

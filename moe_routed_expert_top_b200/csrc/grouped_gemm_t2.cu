@@ -149,7 +149,7 @@ __device__ __forceinline__ void pair_commit(uint32_t bar) {
                : "memory");
 }
 
-// Threads per CTA: producer warp, MMA warp, 4 epilogue warps.
+// Threads per CTA: producer warp, MMA warp, two groups of 4 epilogue warps.
 constexpr int kPairThreads = 320;  // TMA, MMA, two groups of 4 epilogue warps
 
 template <int kMode, int TN, bool kGather>
