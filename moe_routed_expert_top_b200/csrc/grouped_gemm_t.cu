@@ -448,8 +448,10 @@ __global__ void __launch_bounds__(TCfg<kMode, TN>::kThreads, 1)
 #pragma unroll
               for (int k = 0; k < Cfg::K_STEPS; ++k)
                 mma_fp8(d, adesc + 2 * k, bdesc + 2 * k, idesc8, k != 0 ? 1u : 0u);
-              // one commit per K-block: the epilogue, which waits for this
-              // buffer anyway, releases the shared-memory stage when it lands
+              // the stage is released as soon as these MMAs complete, not when
+              // the epilogue gets to this K-block's buffer: the ring keeps its
+              // depth while the epilogue lags
+              mma_commit(empty0 + 8 * stage);
               mma_commit(tfull0 + 8 * acc);
             }
             if (++stage == STAGES) {
@@ -556,7 +558,6 @@ __global__ void __launch_bounds__(TCfg<kMode, TN>::kThreads, 1)
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     int acc = 0;
     uint32_t acc_phase = 0;
-    int stage = 0;  // FP8: the shared-memory stage of the next K-block, as the MMA thread counts
     int sslot = 0;  // FP8: the scale ring's slot of the next tile, and its phase
     uint32_t sphase = 0;
     int ecur = 0;
@@ -583,9 +584,6 @@ __global__ void __launch_bounds__(TCfg<kMode, TN>::kThreads, 1)
             ok = false;
             break;
           }
-          // this K-block's MMAs have completed: its shared-memory stage is free
-          if (grp == 0 && et == 0) mbar_arrive(empty0 + 8 * stage);
-          if (++stage == STAGES) stage = 0;
           tc_fence_after();
           if (mine) {
             const uint32_t tbk = lane_base + static_cast<uint32_t>(acc * TN + grp * 32);
