@@ -41,7 +41,7 @@ struct DualCfg {
   static constexpr int NS = 3;
   static constexpr int ROW_BYTES = 272;
   static constexpr int IN_BYTES = 128 * ROW_BYTES;
-  static constexpr int RED_BYTES = 256 * 8;  // per-tile column maxima: 4 x 64 float2
+  static constexpr int RED_BYTES = 512 * 8;  // per-tile column maxima: 2 slots x 4 x 64 float2
   static constexpr int META_TILES = 512;  // tiles per CTA with precomputed rows
   static constexpr int SMEM = NS * IN_BYTES + RED_BYTES + META_TILES * 8;
 };
@@ -323,13 +323,13 @@ __global__ void __launch_bounds__(kPlainThreads, 2) quant_dual_kernel(const Dual
       a0 = a1 = red[stage];
       if (t == 0) red[stage == 0 ? 2 : stage - 1] = 0.0f;  // slot of tile j + 2
     } else {
-      const uint32_t mx = absmax_tree<32>(wd);
-      reinterpret_cast<float2*>(red)[tq * 64 + cp] = make_float2(absmax_lo(mx), absmax_hi(mx));
-      __syncthreads();
+      // the column maxima of this tile's four token quarters, left in slot
+      // j & 1 by colmax_pass one barrier earlier
+      const float2* slot = reinterpret_cast<const float2*>(red) + (j & 1) * 256;
       a0 = a1 = 0.0f;
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const float2 q2 = reinterpret_cast<const float2*>(red)[k * 64 + cp];
+        const float2 q2 = slot[k * 64 + cp];
         a0 = fmaxf(a0, q2.x);
         a1 = fmaxf(a1, q2.y);
       }
@@ -356,11 +356,27 @@ __global__ void __launch_bounds__(kPlainThreads, 2) quant_dual_kernel(const Dual
     }
   };
 
+  // Per-tile scales: each thread's maxima of columns 2cp, 2cp+1 over its 32
+  // tokens of tile j, into slot j & 1, one barrier before tile j's column
+  // pass reads the four token quarters' values.
+  auto colmax_pass = [&](int j, int stage) {
+    const uint8_t* st = smem_raw + stage * C::IN_BYTES + tq * 32 * C::ROW_BYTES + coff;
+    uint32_t wd[32];
+#pragma unroll
+    for (int r = 0; r < 32; ++r) wd[r] = *reinterpret_cast<const uint32_t*>(st + r * C::ROW_BYTES);
+    const uint32_t mx = absmax_tree<32>(wd);
+    reinterpret_cast<float2*>(red)[(j & 1) * 256 + tq * 64 + cp] =
+        make_float2(absmax_lo(mx), absmax_hi(mx));
+  };
+
   issue(0, 0);
   issue(1, 1);
   cp_async_wait<1>();  // tile 0 has landed
   __syncthreads();
-  if (n_my > 0) row_pass(0, 0);
+  if (n_my > 0) {
+    row_pass(0, 0);
+    if constexpr (!kTransBlock) colmax_pass(0, 0);
+  }
   int stage = 0;  // stage (and block-amax slot) of tile j: j mod 3
   for (int j = 0; j + 1 < n_my; ++j) {
     cp_async_wait<0>();  // tile j + 1 has landed
@@ -369,6 +385,7 @@ __global__ void __launch_bounds__(kPlainThreads, 2) quant_dual_kernel(const Dual
     const int s2 = s1 == 2 ? 0 : s1 + 1;
     issue(j + 2, s2);  // into the stage column pass j - 1 released
     row_pass(j + 1, s1);
+    if constexpr (!kTransBlock) colmax_pass(j + 1, s1);
     col_pass(j, stage);
     stage = s1;
   }
