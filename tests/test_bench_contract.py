@@ -59,3 +59,45 @@ def test_gpus_flag_must_match_the_launchers_world_size():
                        capture_output=True, text=True, cwd=ROOT, timeout=600, env=env)
     assert r.returncode != 0
     assert "must agree" in r.stderr
+
+
+def _bench_module():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def test_work_model_bytes_match_the_workload_sizes():
+    """The algorithmic bytes behind every roofline figure, against the sizes the
+    workloads fix: x_perm of Qwen3 / DeepSeek-V3 prefill is 134 / 470 MB
+    (P x H bf16), Qwen3's touched gate+up weights 805.3 MB, and y leaves the
+    down GEMM as f16e (2 bytes per value plus one exponent byte per 128)."""
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    from moe_inputs import get_config
+    b = _bench_module()
+    for name, xperm_mb in (("qwen3_prefill", 134.2), ("dsv3_prefill", 469.8)):
+        cfg = get_config(name)
+        ids = np.arange(cfg.T * cfg.top_k).reshape(cfg.T, cfg.top_k) % cfg.E  # every expert
+        wm = b.work_model(cfg, ids)
+        P = cfg.T * cfg.top_k
+        assert wm["touched"] == cfg.E
+        assert abs(P * cfg.H * 2 / 1e6 - xperm_mb) < 0.1
+        w_gu = cfg.E * 2 * cfg.F * cfg.H * 2
+        assert wm["gate_up_bytes"] == w_gu + P * cfg.H * 2 + P * cfg.F * 2
+        assert wm["down_bytes"] == cfg.E * cfg.H * cfg.F * 2 + P * cfg.F * 2 + P * cfg.H * 2 + P * (cfg.H // 128)
+        assert wm["gate_up_flops"] == 4.0 * P * cfg.H * cfg.F
+        assert wm["flops"] == 6.0 * P * cfg.H * cfg.F + 6.0 * cfg.T * cfg.H * cfg.F_shared
+    cfg = get_config("qwen3_decode")
+    ids = np.arange(cfg.T * cfg.top_k).reshape(cfg.T, cfg.top_k) % cfg.E
+    assert abs(b.work_model(cfg, ids)["gate_up_bytes"] - 4096 * 2048 * 2 - 4096 * 768 * 2
+               - 805.306368e6) < 1
+    # FP8 down: e4m3 weights and their 128x128 block scales, e4m3 h
+    cfg = get_config("dsv3_decode_fp8")
+    ids = np.arange(cfg.T * cfg.top_k).reshape(cfg.T, cfg.top_k) % cfg.E
+    wm = b.work_model(cfg, ids)
+    P = cfg.T * cfg.top_k
+    w_dn = cfg.E * cfg.H * cfg.F + cfg.E * (cfg.H // 128) * (cfg.F // 128) * 4
+    assert wm["down_bytes"] == w_dn + P * cfg.F + P * cfg.H * 2 + P * (cfg.H // 128)
