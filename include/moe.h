@@ -337,7 +337,9 @@ moe_status moe_quantize_weight_128x128(int32_t batch, int32_t N, int32_t K, cons
  * Streams: everything is ordered on `stream`. When F_shared > 0 and the routed
  * experts average at most 64 rows (T*k <= 64*E), the shared expert's two GEMMs
  * run on a second, library-owned stream of the current device (created on first
- * use, never destroyed), forked from `stream` by an event before them and joined
+ * use outside stream capture, never destroyed; while `stream` is being captured
+ * and that stream does not exist yet, they run on `stream`), forked from
+ * `stream` by an event before them and joined
  * back by an event before the unpermute; the routed GEMMs then use the other SMs.
  * Under CUDA graph capture of `stream` the fork and join are graph edges. */
 moe_status moe_experts_forward(const moe_problem* prob, const void* hidden,

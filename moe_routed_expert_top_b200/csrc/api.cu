@@ -57,15 +57,16 @@ moe_status check_problem(const moe_problem* pr, bool need_gemm) {
 int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
 
 // A second stream per device on which the forward runs the shared expert beside
-// the routed GEMMs (created on first use; null if that fails, and the forward
-// then runs everything on the caller's stream).
-cudaStream_t side_stream() {
+// the routed GEMMs (created on first use outside stream capture; null if it
+// does not exist yet and may not be created now, or if creating it fails: the
+// forward then runs everything on the caller's stream).
+cudaStream_t side_stream(bool may_create) {
   static cudaStream_t streams[64] = {};
   static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
   std::lock_guard<std::mutex> lock(mu);
-  if (streams[dev] == nullptr) {
+  if (streams[dev] == nullptr && may_create) {
     cudaStream_t t = nullptr;
     if (cudaStreamCreateWithFlags(&t, cudaStreamNonBlocking) != cudaSuccess) {
       cudaGetLastError();
@@ -529,7 +530,15 @@ moe_status moe_experts_forward(const moe_problem* prob, const void* hidden,
     d.A = hidden;
     d.B = ws_gate_up;
     d.C = base + w.hs;
-    cudaStream_t side = static_cast<int64_t>(T) * k <= 64LL * E ? side_stream() : nullptr;
+    // a stream is not created while the caller's stream is being captured
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) {
+      cudaGetLastError();
+      cap = cudaStreamCaptureStatusActive;
+    }
+    cudaStream_t side = static_cast<int64_t>(T) * k <= 64LL * E
+                            ? side_stream(cap == cudaStreamCaptureStatusNone)
+                            : nullptr;
     beside = side != nullptr && fork.create() && join.create();
     cudaStream_t sst = st;
     if (beside) {

@@ -205,6 +205,48 @@ def test_graph_replay_matches_eager():
     del graph
 
 
+def test_graph_capture_before_any_eager_call():
+    """In a fresh process, the first forward is the one captured into a CUDA
+    graph: the library then creates no stream during the capture and runs the
+    shared expert on the captured stream. The replay equals a later eager call
+    (which uses the side stream) bit for bit."""
+    import subprocess
+    import sys
+    import os
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    script = """
+import sys, torch
+sys.path.insert(0, %r)
+from tests import test_gpu_forward as F
+from moe_routed_expert_top_b200.layer import RoutedExperts
+cfg = next(c for c in F.MID if c.name == "mid_shared_beside")
+hidden, ids, w, weights = F._inputs(cfg)
+layer = RoutedExperts(weights["w_gate_up"], weights["w_down"], cfg.top_k, cfg.score_fn,
+                      cfg.renormalize, cfg.routed_scaling_factor, cfg.down_fp8,
+                      weights.get("ws_gate_up"), weights.get("ws_down"))
+ids_d = torch.from_numpy(ids).cuda()
+w_d = torch.from_numpy(w).cuda()
+out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device="cuda")
+layer.workspace(cfg.T, hidden.device)
+torch.cuda.synchronize()
+g = torch.cuda.CUDAGraph()
+with torch.cuda.graph(g):
+    layer.forward(hidden, ids_d, w_d, out)
+g.replay()
+torch.cuda.synchronize()
+captured = out.clone()
+eager = layer.forward(hidden, ids_d, w_d)
+torch.cuda.synchronize()
+assert layer.device_status() == 0
+assert torch.equal(captured.view(torch.int16), eager.view(torch.int16))
+del g
+print("capture-first ok")
+""" % root
+    r = subprocess.run([sys.executable, "-c", script], capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-4000:]
+    assert "capture-first ok" in r.stdout
+
+
 def test_deterministic_repeat():
     cfg = get_config("tiny", name="det", T=333, E=16, top_k=4, H=256, F=256, seed=35)
     hidden, ids, w, weights = _inputs(cfg)
